@@ -1,0 +1,187 @@
+/*
+ * fca.h -- C ABI of libfca_b200.so: Forest Cascade Attention (FCA) decode on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("ZoRRo Inference & Forest Cascade Attention", sections
+ * "Overview" and "Core Mechanism"): for one decode step of a batch whose paged
+ * KV caches share prefixes,
+ *   1. discover the groups of requests that share a KV-cache prefix
+ *      (fca_plan);
+ *   2. run one grouped pass over each group's shared prefix blocks, so each
+ *      such block is read once per group instead of once per request;
+ *   3. run one pass per request over its own (suffix) blocks;
+ *   4. reduce the partial results by their log-sum-exp weights
+ *      (steps 2-4: fca_decode).
+ * The output equals standard softmax attention over each request's whole
+ * sequence.
+ *
+ * Cache layout ("PagedAttention vs. RadixAttention", "How PagedAttention
+ * Works", steps 1-2 and 4): K and V are bf16 [num_blocks][block_size]
+ * [num_kv_heads][head_dim], row-major; a request's block table row maps its
+ * logical block j to a physical block id.  Two requests share a block when
+ * their tables hold the same physical id at the same logical index.  Only
+ * FULL blocks (j < seq_len / block_size) are shareable; a partly filled block
+ * is treated as private to each request that references it (copy-on-write).
+ *
+ * Conventions for every call:
+ *   - Pointers marked DEVICE are CUDA device pointers on the current device;
+ *     HOST pointers are ordinary host memory.  The caller owns every buffer it
+ *     passes in; the library owns only what a plan handle holds.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls that
+ *     take a stream are asynchronous on it unless stated otherwise.
+ *   - Functions return fca_status; nothing throws, traps or aborts across the
+ *     ABI.  On an error return no output has been written unless stated.
+ *   - Query head h reads KV head h / (num_q_heads / num_kv_heads).
+ *   - lse is the natural-log log-sum-exp of the scaled scores, fp32.
+ */
+#ifndef FCA_H_
+#define FCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fca_status {
+    FCA_OK = 0,
+    FCA_ERR_INVALID_ARG = 1,   /* bad shape, null pointer, seq_len out of range */
+    FCA_ERR_BAD_BLOCK_ID = 2,  /* a referenced table entry is outside [0, num_blocks) */
+    FCA_ERR_UNSUPPORTED = 3,   /* valid input this build does not handle (e.g. head_dim) */
+    FCA_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+    FCA_ERR_OOM = 5,           /* device allocation failed */
+    FCA_ERR_DEVICE_FLAG = 6    /* a kernel reported an internal error (bounded wait ran out) */
+} fca_status;
+
+/* Opaque plan: the group forest, per-request suffix starts, the work lists of
+ * the three passes and the device workspace they need.  Library-owned; free
+ * with fca_plan_destroy.  A plan stays valid for every layer whose caches use
+ * the same block tables and shapes; q/k/v pointers are bound per decode. */
+typedef struct fca_plan_s *fca_plan_t;
+
+/* Plan options.  Pass NULL for the defaults. */
+typedef struct fca_plan_opts {
+    int32_t min_group_size;    /* groups need at least this many requests (>= 2; default 2) */
+    int32_t min_shared_blocks; /* a group shorter than this many blocks is folded into the
+                                  group below it or into its members' suffixes (>= 1; default 1) */
+    int32_t split_tokens;      /* split-KV chunk length in tokens, multiple of 64;
+                                  0 = automatic */
+    int32_t flags;             /* FCA_PLAN_* bits */
+} fca_plan_opts;
+
+/* Build a plan with no groups: every request reads its whole table in its own
+ * pass.  fca_decode on such a plan is the flat (non-cascaded) paged decode. */
+#define FCA_PLAN_FLAT 1u
+
+/* Default options (min_group_size 2, min_shared_blocks 1, split auto, flags 0). */
+void fca_plan_opts_default(fca_plan_opts *opts /* HOST, out */);
+
+/*
+ * fca_plan -- group discovery ("Core Mechanism" step 1) and work-list build.
+ *
+ *   block_tables  DEVICE int32 [num_requests][max_blocks]; entries at
+ *                 j >= ceil(seq_len / block_size) are ignored.
+ *   seq_lens      DEVICE int32 [num_requests]; each in [1, max_blocks*block_size].
+ *   block_size    tokens per block; this build supports 16.
+ *   num_blocks    physical blocks in the caches (ids must be in [0, num_blocks)).
+ *   num_q_heads, num_kv_heads  num_q_heads % num_kv_heads == 0,
+ *                 num_q_heads / num_kv_heads <= 16.
+ *   head_dim      64 or 128.
+ *   out_plan      HOST, out: the new plan (NULL on error).
+ *
+ * Runs GPU kernels on `stream`, then synchronises the stream once to read back
+ * the sizes of the forest and work lists and allocates the plan's device
+ * workspace (cudaMalloc).  The input buffers may be reused once it returns.
+ * Errors: FCA_ERR_INVALID_ARG (shapes, a seq_len out of range),
+ * FCA_ERR_BAD_BLOCK_ID (a referenced id out of range), FCA_ERR_UNSUPPORTED,
+ * FCA_ERR_CUDA, FCA_ERR_OOM.  num_requests <= 65536, max_blocks <= 1 << 20.
+ */
+fca_status fca_plan(const int32_t *block_tables, int32_t max_blocks, const int32_t *seq_lens,
+                    int32_t num_requests, int32_t block_size, int32_t num_blocks,
+                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                    const fca_plan_opts *opts, fca_plan_t *out_plan, void *stream);
+
+/*
+ * fca_decode -- steps 2-4 of "Core Mechanism": the grouped prefix pass, the
+ * per-request suffix pass and the log-sum-exp merge, for one layer.
+ *
+ *   q        DEVICE bf16 [num_requests][num_q_heads][head_dim], 16-byte aligned.
+ *   k_cache, v_cache  DEVICE bf16 [num_blocks][block_size][num_kv_heads][head_dim],
+ *            16-byte aligned.
+ *   out      DEVICE bf16 [num_requests][num_q_heads][head_dim] (round to nearest even).
+ *   lse      DEVICE fp32 [num_requests][num_q_heads], or NULL to skip.
+ *   scale    multiplier of q.k (normally 1/sqrt(head_dim)).
+ *
+ * Asynchronous on `stream`; uses the plan's workspace, so decodes that share
+ * a plan must be ordered on one stream.  A kernel that detects an internal
+ * error records it in the plan; read it with fca_check_device_status.
+ */
+fca_status fca_decode(const void *q, const void *k_cache, const void *v_cache, fca_plan_t plan,
+                      void *out, float *lse, float scale, void *stream);
+
+/*
+ * fca_flat_decode -- the flat paged decode baseline: standard split-KV
+ * attention of every request over its whole table, same kernels and merge.
+ * `plan` must have been built with FCA_PLAN_FLAT (else FCA_ERR_INVALID_ARG).
+ * Arguments as fca_decode.
+ */
+fca_status fca_flat_decode(const void *q, const void *k_cache, const void *v_cache,
+                           fca_plan_t plan, void *out, float *lse, float scale, void *stream);
+
+/* Sizes and byte counts of a plan (HOST struct, filled synchronously). */
+typedef struct fca_plan_stats {
+    int32_t num_requests, num_groups, max_depth, num_q_heads, num_kv_heads, head_dim;
+    int32_t split_tokens;           /* chunk length actually used */
+    int32_t prefix_items, suffix_items;   /* work items of the two passes */
+    int64_t num_partials;           /* partial (o, lse) rows written per decode */
+    int64_t unique_kv_tokens;       /* each referenced physical block once, its valid tokens */
+    int64_t unique_kv_bytes;        /* unique_kv_tokens * num_kv_heads * head_dim * 2 * 2 */
+    int64_t flat_kv_bytes;          /* sum of seq_len * num_kv_heads * head_dim * 2 * 2 */
+    int64_t fca_kv_bytes;           /* KV bytes the FCA passes read (prefix once per group) */
+    int64_t workspace_bytes;        /* device bytes the plan holds */
+} fca_plan_stats;
+
+fca_status fca_plan_get_stats(fca_plan_t plan, fca_plan_stats *stats /* HOST, out */);
+
+/*
+ * fca_plan_export -- copy the canonical forest to HOST buffers (synchronous).
+ * Canonical order: groups by (first block ascending, smallest member
+ * ascending); members of a group ascending; parent as an index in that order
+ * (-1 for a root).  Group g reads blocks [a[g], b[g]) of its members' tables;
+ * its members are members[member_off[g] .. member_off[g] + n_members[g]).
+ * suffix_start[r] is the first block of request r's own pass (the b of its
+ * deepest group, else 0).  Any output pointer may be NULL.  Capacities:
+ * num_groups entries for the group arrays, the total member count for
+ * members, num_requests for suffix_start (see fca_plan_get_stats and
+ * fca_plan_member_count).
+ */
+fca_status fca_plan_export(fca_plan_t plan, int32_t *a, int32_t *b, int32_t *parent,
+                           int32_t *member_off, int32_t *n_members, int32_t *members,
+                           int32_t *suffix_start);
+
+/* Total member entries over all groups (HOST out). */
+fca_status fca_plan_member_count(fca_plan_t plan, int64_t *count);
+
+/* Free a plan and its device workspace (synchronises the device). NULL is ok. */
+fca_status fca_plan_destroy(fca_plan_t plan);
+
+/*
+ * Read and clear the plan's device error word after the work queued on
+ * `stream` finishes (synchronises the stream).  *code (HOST, may be NULL)
+ * receives the raw word: 0 = no error.  Returns FCA_ERR_DEVICE_FLAG when the
+ * word was non-zero.
+ */
+fca_status fca_check_device_status(fca_plan_t plan, void *stream, int32_t *code);
+
+/* Static description of a status code. */
+const char *fca_status_string(fca_status status);
+
+/* Library version string, e.g. "fca_b200 0.1.0 sm_100a". */
+const char *fca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FCA_H_ */
