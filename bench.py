@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of one FCA decode step (one layer) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fca|reference]
+                    [--config llama8b|longctx|forest|mixed|tiny]
+
+A step is one pass of the whole hot path -- grouped prefix pass, per-request
+pass, log-sum-exp merge -- over the configuration's synthetic batch, with the
+plan built beforehand (plan time is reported separately).  Inputs are
+resident in HBM; L2 is flushed (256 MiB write) before every timed step.
+Every step is timed on the device with CUDA events on the launching stream,
+per pass; ms_per_step is the mean over the K timed steps (max over ranks).
+
+value = unique KV bytes processed by all ranks per step / ms_per_step, in
+GB/s (each shared block counted once).  Under torchrun every rank decodes its
+own independent batch (seed = rank): weak scaling, no collective on the data
+path; the only collectives are the barriers and the max-reduction of the
+timings.
+
+Extra keys: the flat paged decode of the same batch (speedup_vs_flat), the
+per-kernel roofline of the dominant kernel, the CPU oracle as a baseline, an
+end-to-end number through the public API with host buffers, and the SM clocks
+sampled during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FCA decode µs/step; unique-KV HBM GB/s (% peak); speedup vs flat paged decode"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+DOMINANT_SOURCES = {"prefix": "fca_prefix.cu", "suffix": "fca_suffix.cu", "merge": "fca_merge.cu"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["fca", "reference"], default="fca")
+    ap.add_argument("--config", default="llama8b")
+    ap.add_argument("--split", type=int, default=0, help="split-KV chunk tokens (0 = automatic)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-flat", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0,
+                    help="approximate CPU seconds of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_desc(w):
+    return (f"{w.name}: {w.description}; {w.R} requests, heads {w.Hq}/{w.Hkv}/{w.D}, bf16 paged "
+            f"KV, block {w.block_size}, {w.num_blocks} physical blocks")
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        loaded = [s for s, p in zip(sm, pw) if p >= 200.0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(pw) if pw else None}
+
+
+def gpu_id_for(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ------------------------------------------------------------------ oracle legs
+
+def oracle_sample(w, budget_s: float, seed: int = 0):
+    """Time the oracle (as it stands) on whole requests, all heads, until about
+    budget_s seconds of work; return (seconds, tokens covered, requests)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(w.R)
+    # calibrate on one request
+    r0 = int(order[0])
+    pairs = np.array([[r0, h] for h in range(w.Hq)], np.int32)
+    t = time.perf_counter()
+    oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, pairs=pairs)
+    t1 = max(time.perf_counter() - t, 1e-4)
+    per_token = t1 / float(w.seq_lens[r0])
+    target_tokens = budget_s / per_token
+    chosen, tok = [], 0
+    for r in order:
+        chosen.append(int(r))
+        tok += int(w.seq_lens[r])
+        if tok >= target_tokens:
+            break
+    pairs = np.array([[r, h] for r in chosen for h in range(w.Hq)], np.int32)
+    t = time.perf_counter()
+    oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, pairs=pairs)
+    return time.perf_counter() - t, tok, len(chosen)
+
+
+def cpu_cores() -> int:
+    v = os.environ.get("OMP_NUM_THREADS")
+    if v and v.isdigit():
+        return int(v)
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def unique_bytes(w) -> int:
+    import oracle
+    return oracle.unique_kv_tokens(w.block_tables, w.seq_lens, w.block_size, w.num_blocks) * w.Hkv * w.D * 4
+
+
+def reference_arm(args):
+    import fca_workloads
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = fca_workloads.make(args.config, seed=0)
+    ub = unique_bytes(w)
+    total_tok = int(w.seq_lens.sum())
+    per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    times = []
+    for i in range(args.warmup + args.steps):
+        sec, tok, nreq = oracle_sample(w, per_step_budget, seed=i)
+        if i >= args.warmup:
+            times.append(sec * total_tok / tok)   # extrapolated to the whole batch
+    step_s = statistics.mean(times)
+    value = ub / step_s / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(w)}, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": f"whole requests (all {w.Hq} heads) totalling about "
+                                       f"{per_step_budget:.1f} s of CPU work per step, time scaled "
+                                       f"to the full batch of {total_tok} tokens"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ FCA arm
+
+def traffic_record(dominant: str, workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+    or None when there is none for this kernel source and workload."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        ent = rec[dominant][workload]
+        src = os.path.join(ROOT, "shared_prefix_kv_fca_b200", "csrc", DOMINANT_SOURCES[dominant])
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if ent.get("source_sha256_16") != digest:
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def fca_arm(args):
+    import torch
+    import torch.distributed as dist
+
+    import fca_workloads
+    import shared_prefix_kv_fca_b200 as fca
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    w = fca_workloads.make(args.config, seed=rank)
+    q, k, v, bt, sl = w.torch_inputs(dev)
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(w.R, w.Hq, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    plan = fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, split_tokens=args.split)
+    torch.cuda.synchronize(dev)
+    plan_ms = (time.perf_counter() - t0) * 1e3
+    st = plan.stats()
+    flat_plan = None if args.no_flat else fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, flat=True,
+                                                       split_tokens=args.split)
+
+    def run_steps(p, n, timed):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            e = ev[i]
+            e[0].record(stream)
+            fca.fca_prefix_pass(q, k, v, p, w.scale, stream)
+            e[1].record(stream)
+            fca.fca_suffix_pass(q, k, v, p, w.scale, stream)
+            e[2].record(stream)
+            fca.fca_merge_pass(p, out, lse, stream)
+            e[3].record(stream)
+        torch.cuda.synchronize(dev)
+        if not timed:
+            return None
+        per = {"prefix": [], "suffix": [], "merge": [], "step": []}
+        for e in ev:
+            per["prefix"].append(e[0].elapsed_time(e[1]))
+            per["suffix"].append(e[1].elapsed_time(e[2]))
+            per["merge"].append(e[2].elapsed_time(e[3]))
+            per["step"].append(e[0].elapsed_time(e[3]))
+        return {key: statistics.mean(vals) for key, vals in per.items()}
+
+    # ---- FCA, timed region
+    run_steps(plan, args.warmup, False)
+    sampler = ClockSampler(gpu_id_for(local)) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    fca_t = run_steps(plan, args.steps, True)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    barrier()
+    assert fca.fca_check_device_status(plan, stream) == 0
+    step_ms = max_over_ranks(fca_t["step"])
+    n_launch = (1 if (st["prefix_items"] > 0) else 0) + (1 if st["suffix_items"] > 0 else 0) + 1
+
+    # ---- flat paged decode of the same batch
+    flat_ms = None
+    if flat_plan is not None:
+        run_steps(flat_plan, args.warmup, False)
+        barrier()
+        flat_t = run_steps(flat_plan, args.steps, True)
+        barrier()
+        flat_ms = max_over_ranks(flat_t["step"])
+        assert fca.fca_check_device_status(flat_plan, stream) == 0
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        q_h = q.cpu().pin_memory()
+        bt_h = bt.cpu().pin_memory()
+        sl_h = sl.cpu().pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        q_d, bt_d, sl_d = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(sl)
+
+        def e2e_step():
+            q_d.copy_(q_h, non_blocking=True)
+            bt_d.copy_(bt_h, non_blocking=True)
+            sl_d.copy_(sl_h, non_blocking=True)
+            with fca.fca_plan(bt_d, sl_d, w.num_blocks, w.Hq, w.Hkv, w.D, split_tokens=args.split) as p:
+                fca.fca_decode(q_d, k, v, p, out, lse, w.scale, stream)
+                out_h.copy_(out, non_blocking=True)
+                lse_h.copy_(lse, non_blocking=True)
+                torch.cuda.synchronize(dev)
+
+        for _ in range(max(1, args.warmup)):
+            flush.zero_()
+            e2e_step()
+        barrier()
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        e2e_ms = max_over_ranks(statistics.mean(times))
+        h2d = q.numel() * 2 + bt.numel() * 4 + sl.numel() * 4
+        d2h = out.numel() * 2 + lse.numel() * 4
+        e2e = {"value": sum_over_ranks(st["unique_kv_bytes"]) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "includes": "H2D of q and block tables, fca_plan (one host sync), fca_decode, "
+                           "D2H of out and lse; the KV cache is resident state"}
+
+    total_unique = sum_over_ranks(st["unique_kv_bytes"])
+    peak, peak_kind = peaks()
+    value = total_unique / (step_ms * 1e-3) / 1e9
+
+    # dominant kernel and its roofline
+    pass_ms = {key: max_over_ranks(fca_t[key]) for key in ("prefix", "suffix", "merge")}
+    dominant = max(pass_ms, key=pass_ms.get)
+    alg_bytes = {"prefix": st["prefix_kv_bytes"], "suffix": st["suffix_kv_bytes"],
+                 "merge": st["num_partials"] * (w.D + 1) * 4 + w.R * w.Hq * (w.D * 2 + 4)}
+    achieved = alg_bytes[dominant] / (pass_ms[dominant] * 1e-3) / 1e9
+    traffic = traffic_record(dominant, args.config)
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            sec, tok, nreq = oracle_sample(w, args.cpu_budget_s)
+            full_s = sec * float(w.seq_lens.sum()) / tok
+            cpu = {"value": st["unique_kv_bytes"] / full_s / 1e9, "unit": "GB/s", "cores": cpu_cores(),
+                   "kind": "oracle", "ms_per_step": full_s * 1e3,
+                   "sample": f"{nreq} whole requests x {w.Hq} heads ({tok} tokens of "
+                             f"{int(w.seq_lens.sum())}) in {sec:.1f} s, scaled to the full batch"}
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "us_per_step": step_ms * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; per-rank seed = rank)",
+            "config": {"workload": workload_desc(w), "l2": "flushed before every step (256 MiB write)",
+                       "split_tokens": st["split_tokens"], "groups": st["num_groups"],
+                       "unique_kv_bytes_per_rank": st["unique_kv_bytes"],
+                       "flat_kv_bytes_per_rank": st["flat_kv_bytes"], "replicas": world},
+            "pct_of_peak": 100.0 * value / (peak * world), "peak_gbs": peak, "peak_kind": peak_kind,
+            "plan_ms": plan_ms,
+            "passes_us": {key: val * 1e3 for key, val in pass_ms.items()},
+            "flat_us_per_step": flat_ms * 1e3 if flat_ms else None,
+            "speedup_vs_flat": (flat_ms / step_ms) if flat_ms else None,
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_bytes": alg_bytes[dominant],
+                         "peak_note": f"{peak_kind} copy bandwidth (MEASURED_PEAKS hbm_gbs)"},
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": n_launch * args.steps, "impl": "fca",
+        }
+        print(json.dumps(line), flush=True)
+
+    plan.close()
+    if flat_plan is not None:
+        flat_plan.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return reference_arm(args)
+    return fca_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -95,7 +95,7 @@ void fca_plan_opts_default(fca_plan_opts *opts /* HOST, out */);
  * workspace (cudaMalloc).  The input buffers may be reused once it returns.
  * Errors: FCA_ERR_INVALID_ARG (shapes, a seq_len out of range),
  * FCA_ERR_BAD_BLOCK_ID (a referenced id out of range), FCA_ERR_UNSUPPORTED,
- * FCA_ERR_CUDA, FCA_ERR_OOM.  num_requests <= 65536, max_blocks <= 1 << 20.
+ * FCA_ERR_CUDA, FCA_ERR_OOM.  num_requests <= 16384, max_blocks <= 1 << 20.
  */
 fca_status fca_plan(const int32_t *block_tables, int32_t max_blocks, const int32_t *seq_lens,
                     int32_t num_requests, int32_t block_size, int32_t num_blocks,
@@ -129,6 +129,21 @@ fca_status fca_decode(const void *q, const void *k_cache, const void *v_cache, f
 fca_status fca_flat_decode(const void *q, const void *k_cache, const void *v_cache,
                            fca_plan_t plan, void *out, float *lse, float scale, void *stream);
 
+/*
+ * The three passes of fca_decode as separate calls, in the order fca_decode
+ * runs them: fca_prefix_pass (grouped pass over shared prefix blocks, no-op
+ * for a flat plan or a plan without groups), fca_suffix_pass (per-request
+ * pass over own blocks) and fca_merge_pass (log-sum-exp reduction into out
+ * and lse).  Running the three in order on one stream is exactly fca_decode;
+ * they exist so that each kernel can be timed on its own stream.  The first
+ * two write only the plan's partial buffers.  Arguments as fca_decode.
+ */
+fca_status fca_prefix_pass(const void *q, const void *k_cache, const void *v_cache, fca_plan_t plan,
+                           float scale, void *stream);
+fca_status fca_suffix_pass(const void *q, const void *k_cache, const void *v_cache, fca_plan_t plan,
+                           float scale, void *stream);
+fca_status fca_merge_pass(fca_plan_t plan, void *out, float *lse, void *stream);
+
 /* Sizes and byte counts of a plan (HOST struct, filled synchronously). */
 typedef struct fca_plan_stats {
     int32_t num_requests, num_groups, max_depth, num_q_heads, num_kv_heads, head_dim;
@@ -139,6 +154,8 @@ typedef struct fca_plan_stats {
     int64_t unique_kv_bytes;        /* unique_kv_tokens * num_kv_heads * head_dim * 2 * 2 */
     int64_t flat_kv_bytes;          /* sum of seq_len * num_kv_heads * head_dim * 2 * 2 */
     int64_t fca_kv_bytes;           /* KV bytes the FCA passes read (prefix once per group) */
+    int64_t prefix_kv_bytes;        /* of which the grouped pass reads */
+    int64_t suffix_kv_bytes;        /* of which the per-request pass reads */
     int64_t workspace_bytes;        /* device bytes the plan holds */
 } fca_plan_stats;
 

@@ -1,0 +1,290 @@
+"""Forest Cascade Attention (FCA) decode on B200 -- Python binding.
+
+A thin ctypes layer over ``libfca_b200.so`` (C ABI in ``include/fca.h``):
+the functions below carry the C names and only marshal arguments (torch CUDA
+tensors -> device pointers, CUDA streams -> handles).  Every step of the
+decode runs in the library's CUDA kernels; there is no Python or CPU
+fallback, and using any of these calls without the built library raises.
+
+    plan = fca_plan(block_tables, seq_lens, num_blocks, Hq, Hkv, D)
+    fca_decode(q, k_cache, v_cache, plan, out, lse, scale)
+    fca_plan_destroy(plan)
+
+The method ("ZoRRo Inference & Forest Cascade Attention", "Core Mechanism"):
+group discovery over the requests' block tables, one grouped pass per group
+over its shared prefix blocks, one pass per request over its own blocks, and
+a log-sum-exp weighted merge; equal to standard attention.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+__all__ = [
+    "FcaError", "Plan", "fca_plan", "fca_decode", "fca_flat_decode", "fca_plan_get_stats",
+    "fca_plan_export", "fca_plan_member_count", "fca_plan_destroy", "fca_check_device_status",
+    "fca_status_string", "fca_version", "fca_plan_opts_default", "library_path", "load_library",
+    "fca_prefix_pass", "fca_suffix_pass", "fca_merge_pass",
+    "FCA_PLAN_FLAT", "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libfca_b200.so")
+_lib = None
+
+FCA_PLAN_FLAT = 1
+STATUS = {0: "FCA_OK", 1: "FCA_ERR_INVALID_ARG", 2: "FCA_ERR_BAD_BLOCK_ID", 3: "FCA_ERR_UNSUPPORTED",
+          4: "FCA_ERR_CUDA", 5: "FCA_ERR_OOM", 6: "FCA_ERR_DEVICE_FLAG"}
+
+
+class FcaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({fca_status_string(status)})")
+
+
+class fca_plan_opts(ctypes.Structure):
+    _fields_ = [("min_group_size", ctypes.c_int32), ("min_shared_blocks", ctypes.c_int32),
+                ("split_tokens", ctypes.c_int32), ("flags", ctypes.c_int32)]
+
+
+class fca_plan_stats(ctypes.Structure):
+    _fields_ = [("num_requests", ctypes.c_int32), ("num_groups", ctypes.c_int32),
+                ("max_depth", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("split_tokens", ctypes.c_int32), ("prefix_items", ctypes.c_int32),
+                ("suffix_items", ctypes.c_int32), ("num_partials", ctypes.c_int64),
+                ("unique_kv_tokens", ctypes.c_int64), ("unique_kv_bytes", ctypes.c_int64),
+                ("flat_kv_bytes", ctypes.c_int64), ("fca_kv_bytes", ctypes.c_int64),
+                ("prefix_kv_bytes", ctypes.c_int64), ("suffix_kv_bytes", ctypes.c_int64),
+                ("workspace_bytes", ctypes.c_int64)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libfca_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m shared_prefix_kv_fca_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    lib.fca_plan_opts_default.argtypes = [ctypes.POINTER(fca_plan_opts)]
+    lib.fca_plan_opts_default.restype = None
+    lib.fca_plan.argtypes = [vp, i32, vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(fca_plan_opts),
+                             ctypes.POINTER(vp), vp]
+    lib.fca_plan.restype = ctypes.c_int
+    lib.fca_decode.argtypes = [vp, vp, vp, vp, vp, vp, f32, vp]
+    lib.fca_decode.restype = ctypes.c_int
+    lib.fca_flat_decode.argtypes = [vp, vp, vp, vp, vp, vp, f32, vp]
+    lib.fca_flat_decode.restype = ctypes.c_int
+    lib.fca_prefix_pass.argtypes = [vp, vp, vp, vp, f32, vp]
+    lib.fca_prefix_pass.restype = ctypes.c_int
+    lib.fca_suffix_pass.argtypes = [vp, vp, vp, vp, f32, vp]
+    lib.fca_suffix_pass.restype = ctypes.c_int
+    lib.fca_merge_pass.argtypes = [vp, vp, vp, vp]
+    lib.fca_merge_pass.restype = ctypes.c_int
+    lib.fca_plan_get_stats.argtypes = [vp, ctypes.POINTER(fca_plan_stats)]
+    lib.fca_plan_get_stats.restype = ctypes.c_int
+    lib.fca_plan_export.argtypes = [vp, i32p, i32p, i32p, i32p, i32p, i32p, i32p]
+    lib.fca_plan_export.restype = ctypes.c_int
+    lib.fca_plan_member_count.argtypes = [vp, ctypes.POINTER(ctypes.c_int64)]
+    lib.fca_plan_member_count.restype = ctypes.c_int
+    lib.fca_plan_destroy.argtypes = [vp]
+    lib.fca_plan_destroy.restype = ctypes.c_int
+    lib.fca_check_device_status.argtypes = [vp, vp, i32p]
+    lib.fca_check_device_status.restype = ctypes.c_int
+    lib.fca_status_string.argtypes = [ctypes.c_int]
+    lib.fca_status_string.restype = ctypes.c_char_p
+    lib.fca_version.argtypes = []
+    lib.fca_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    return int(t.data_ptr())
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != 0:
+        raise FcaError(rc, where)
+
+
+def fca_status_string(status: int) -> str:
+    return load_library().fca_status_string(int(status)).decode()
+
+
+def fca_version() -> str:
+    return load_library().fca_version().decode()
+
+
+def fca_plan_opts_default() -> fca_plan_opts:
+    o = fca_plan_opts()
+    load_library().fca_plan_opts_default(ctypes.byref(o))
+    return o
+
+
+def fca_plan(block_tables, seq_lens, num_blocks: int, num_q_heads: int, num_kv_heads: int,
+             head_dim: int, block_size: int = 16, min_group_size: int = 2,
+             min_shared_blocks: int = 1, split_tokens: int = 0, flat: bool = False,
+             stream=None) -> "Plan":
+    """Group discovery + work lists.  block_tables int32 [R, max_blocks] and
+    seq_lens int32 [R] are CUDA tensors."""
+    lib = load_library()
+    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens")):
+        if not t.is_cuda or str(t.dtype) != "torch.int32" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    R, mb = block_tables.shape
+    o = fca_plan_opts(min_group_size, min_shared_blocks, split_tokens, FCA_PLAN_FLAT if flat else 0)
+    handle = ctypes.c_void_p()
+    rc = lib.fca_plan(_ptr(block_tables), mb, _ptr(seq_lens), R, block_size, num_blocks, num_q_heads,
+                      num_kv_heads, head_dim, ctypes.byref(o), ctypes.byref(handle),
+                      _stream_handle(stream))
+    _check(rc, "fca_plan")
+    return Plan(handle, R, num_q_heads, num_kv_heads, head_dim, flat)
+
+
+def _decode(fn_name: str, q, k_cache, v_cache, plan: "Plan", out, lse, scale, stream) -> None:
+    lib = load_library()
+    if scale is None:
+        scale = 1.0 / math.sqrt(plan.head_dim)
+    for t, name in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (out, "out")):
+        if not t.is_cuda or str(t.dtype) != "torch.bfloat16" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if lse is not None and (str(lse.dtype) != "torch.float32" or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 CUDA tensor")
+    rc = getattr(lib, fn_name)(_ptr(q), _ptr(k_cache), _ptr(v_cache), plan.handle, _ptr(out),
+                               _ptr(lse), float(scale), _stream_handle(stream))
+    _check(rc, fn_name)
+
+
+def fca_decode(q, k_cache, v_cache, plan: "Plan", out, lse=None, scale=None, stream=None) -> None:
+    """Grouped prefix pass + per-request pass + LSE merge into out (and lse)."""
+    _decode("fca_decode", q, k_cache, v_cache, plan, out, lse, scale, stream)
+
+
+def fca_flat_decode(q, k_cache, v_cache, plan: "Plan", out, lse=None, scale=None,
+                    stream=None) -> None:
+    """Flat (non-cascaded) paged decode; plan must be built with flat=True."""
+    _decode("fca_flat_decode", q, k_cache, v_cache, plan, out, lse, scale, stream)
+
+
+def fca_prefix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) -> None:
+    """Grouped pass over shared prefix blocks only (writes the plan's partials)."""
+    scale = 1.0 / math.sqrt(plan.head_dim) if scale is None else scale
+    _check(load_library().fca_prefix_pass(_ptr(q), _ptr(k_cache), _ptr(v_cache), plan.handle,
+                                          float(scale), _stream_handle(stream)), "fca_prefix_pass")
+
+
+def fca_suffix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) -> None:
+    """Per-request pass over own blocks only (writes the plan's partials)."""
+    scale = 1.0 / math.sqrt(plan.head_dim) if scale is None else scale
+    _check(load_library().fca_suffix_pass(_ptr(q), _ptr(k_cache), _ptr(v_cache), plan.handle,
+                                          float(scale), _stream_handle(stream)), "fca_suffix_pass")
+
+
+def fca_merge_pass(plan: "Plan", out, lse=None, stream=None) -> None:
+    """Log-sum-exp merge of the plan's partials into out (and lse)."""
+    _check(load_library().fca_merge_pass(plan.handle, _ptr(out), _ptr(lse), _stream_handle(stream)),
+           "fca_merge_pass")
+
+
+def fca_plan_get_stats(plan: "Plan") -> dict:
+    st = fca_plan_stats()
+    _check(load_library().fca_plan_get_stats(plan.handle, ctypes.byref(st)), "fca_plan_get_stats")
+    return {name: getattr(st, name) for name, _ in fca_plan_stats._fields_}
+
+
+def fca_plan_member_count(plan: "Plan") -> int:
+    n = ctypes.c_int64()
+    _check(load_library().fca_plan_member_count(plan.handle, ctypes.byref(n)),
+           "fca_plan_member_count")
+    return int(n.value)
+
+
+def fca_plan_export(plan: "Plan") -> dict:
+    """Canonical forest as numpy int32 arrays (synchronises the device)."""
+    import numpy as np
+    st = fca_plan_get_stats(plan)
+    ng, R = st["num_groups"], st["num_requests"]
+    nm = fca_plan_member_count(plan)
+    arr = {k: np.zeros(max(ng, 1), np.int32) for k in ("a", "b", "parent", "member_off", "n_members")}
+    arr["members"] = np.zeros(max(nm, 1), np.int32)
+    arr["suffix_start"] = np.zeros(R, np.int32)
+
+    def p(a):
+        return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    rc = load_library().fca_plan_export(plan.handle, p(arr["a"]), p(arr["b"]), p(arr["parent"]),
+                                        p(arr["member_off"]), p(arr["n_members"]),
+                                        p(arr["members"]), p(arr["suffix_start"]))
+    _check(rc, "fca_plan_export")
+    for k in ("a", "b", "parent", "member_off", "n_members"):
+        arr[k] = arr[k][:ng]
+    arr["members"] = arr["members"][:nm]
+    return arr
+
+
+def fca_check_device_status(plan: "Plan", stream=None) -> int:
+    """Raw device error word (0 = fine); raises FcaError when it is set."""
+    code = ctypes.c_int32()
+    rc = load_library().fca_check_device_status(plan.handle, _stream_handle(stream),
+                                                ctypes.byref(code))
+    if rc not in (0, 6):
+        _check(rc, "fca_check_device_status")
+    if rc == 6:
+        raise FcaError(rc, f"fca_check_device_status (word {code.value:#x})")
+    return int(code.value)
+
+
+def fca_plan_destroy(plan: "Plan") -> None:
+    plan.close()
+
+
+class Plan:
+    """Owner of an fca_plan_t handle."""
+
+    def __init__(self, handle: ctypes.c_void_p, R: int, Hq: int, Hkv: int, D: int, flat: bool):
+        self.handle = handle
+        self.num_requests, self.num_q_heads, self.num_kv_heads, self.head_dim = R, Hq, Hkv, D
+        self.flat = flat
+
+    def stats(self) -> dict:
+        return fca_plan_get_stats(self)
+
+    def export(self) -> dict:
+        return fca_plan_export(self)
+
+    def close(self) -> None:
+        if self.handle is not None and self.handle.value:
+            _check(load_library().fca_plan_destroy(self.handle), "fca_plan_destroy")
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()

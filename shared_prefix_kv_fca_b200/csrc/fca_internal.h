@@ -1,0 +1,106 @@
+// Internal declarations shared by the host and device parts of libfca_b200.
+//
+// Work-list records and the plan object.  Nothing here is part of the C ABI
+// (include/fca.h); the layout of these records may change between builds.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fca.h"
+
+namespace fca {
+
+constexpr int kBlockSize = 16;        // tokens per paged block (the only size built)
+constexpr int kPrefixTileRows = 128;  // stacked query rows per tcgen05 tile (MMA M)
+constexpr int kStageTokens = 64;      // tokens per pipeline stage of the grouped pass
+constexpr int kMaxGqa = 16;           // query heads per KV head handled by the own pass
+constexpr int kMaxRequests = 16384;   // groups are sorted in one CTA's shared memory
+constexpr int kMaxRequestsFallback = 4096;  // all-pairs LCP path (see fca_plan.cu)
+
+// Device error word bits (fca_check_device_status).
+constexpr int32_t kErrWaitTimeout = 1;     // a bounded mbarrier wait ran out
+constexpr int32_t kErrBadItem = 2;         // a work item failed its own range check
+constexpr int32_t kErrPlanInternal = 4;    // a planner consistency check failed (no write done)
+
+// Planner status bits (read back inside fca_plan).
+constexpr int32_t kPlanBadSeqLen = 1;
+constexpr int32_t kPlanBadBlockId = 2;
+constexpr int32_t kPlanInconsistent = 4;   // block ids do not identify prefixes
+constexpr int32_t kPlanTooManyGroups = 8;
+
+// One tile of the grouped prefix pass: rows [row0, row0 + nrows) of group
+// `group`'s stacked queries (member i / G, query head head * G + i % G),
+// against tokens [tok0, tok1) of the table row of request `bt_row`.
+struct PrefixItem {
+    int32_t group, head, row0, nrows;
+    int32_t tok0, tok1, bt_row, part_row0;   // partial row of stacked row row0
+};
+
+// One chunk of a request's own pass: the G query heads of KV head `head`
+// against tokens [tok0, tok1) of request `request`'s table.
+struct SuffixItem {
+    int32_t request, head, tok0, tok1;
+    int32_t part_row0, pad0, pad1, pad2;     // first of G partial rows
+};
+
+// Sizes the planner computes on the device and fca_plan reads back once.
+struct PlanHeader {
+    int32_t status;
+    int32_t n_groups;
+    int32_t n_member_entries;   // sum of group sizes
+    int32_t max_depth;
+    int32_t split_tokens;
+    int32_t n_prefix_items;
+    int32_t n_suffix_items;
+    int32_t n_prefix_partials;  // partial rows written by the grouped pass
+    int32_t n_suffix_partials;
+    int32_t n_chain_entries;    // sum over requests of their group depth
+    int64_t unique_kv_tokens;
+    int64_t fca_kv_tokens;      // token-blocks the FCA passes read (per KV head)
+    int64_t flat_kv_tokens;
+    int64_t prefix_tok_sum;     // sum over groups of their token count
+    int64_t suffix_tok_sum;
+};
+
+}  // namespace fca
+
+// The plan object behind fca_plan_t.
+struct fca_plan_s {
+    int device = 0;
+    int32_t R = 0, max_blocks = 0, block_size = 0, num_blocks = 0;
+    int32_t Hq = 0, Hkv = 0, D = 0, G = 0;
+    fca_plan_opts opts{};
+    bool flat = false;
+    fca::PlanHeader hdr{};
+    size_t workspace_bytes = 0;
+
+    // copies of the inputs
+    int32_t* bt = nullptr;           // [R][max_blocks]
+    int32_t* seq_lens = nullptr;     // [R]
+    // forest, canonical order
+    int32_t* g_a = nullptr;          // [n_groups]
+    int32_t* g_b = nullptr;
+    int32_t* g_parent = nullptr;
+    int32_t* g_moff = nullptr;
+    int32_t* g_nm = nullptr;
+    int32_t* g_nch = nullptr;        // split chunks of the group's token range
+    int32_t* g_part = nullptr;       // partial row of (group, head 0, chunk 0, row 0)
+    int32_t* members = nullptr;      // [n_member_entries]
+    int32_t* suffix_start = nullptr; // [R] blocks
+    int32_t* chain_off = nullptr;    // [R + 1] into chain_g / chain_pos
+    int32_t* chain_g = nullptr;      // groups of request r, root first
+    int32_t* chain_pos = nullptr;    // r's index among the group's members
+    int32_t* s_nch = nullptr;        // [R] chunks of r's own pass
+    int32_t* s_part = nullptr;       // [R] partial row of (r, head 0, chunk 0)
+    fca::PrefixItem* prefix_items = nullptr;
+    fca::SuffixItem* suffix_items = nullptr;
+    float* part_o = nullptr;         // [n_partials][D]
+    float* part_lse = nullptr;       // [n_partials]
+    int32_t* dev_status = nullptr;   // device error word
+
+    // every cudaMalloc the plan owns (freed by fca_plan_destroy)
+    std::vector<void*> dev_allocs;
+};

@@ -1,0 +1,875 @@
+// Group discovery and work-list construction for Forest Cascade Attention.
+//
+// "ZoRRo Inference & Forest Cascade Attention", "Core Mechanism" step 1:
+// discover the groups of requests that share a KV-cache prefix.  Sharing is
+// by physical block: requests that start with the same prompt reference the
+// same physical blocks ("PagedAttention vs. RadixAttention", "How
+// PagedAttention Works", step 4), and only full blocks are shareable (a block
+// that is still being written is copied before it diverges).
+//
+// The forest is the trie of the requests' full-block id sequences: a node is
+// a prefix, its member set is the requests whose tables start with it, and a
+// group is a maximal run of depths over which the member set does not change
+// (and has at least min_group_size members).
+//
+// Fast path (every table produced by a prefix-caching allocator).  A trie node
+// at depth k + 1 is identified by the physical block at logical index k,
+// because a cached block's identity already stands for its whole prefix
+// ("How vLLM Implements Prefix Caching": each block's hash chains its parent's
+// hash, so equal blocks imply equal prefixes).  The planner checks that
+// property on the device -- every block id appears at one logical index only,
+// and all requests holding block b at index k hold the same block at k - 1 --
+// which makes "same block at index k" equivalent to "same prefix of length
+// k + 1".  Then a node's member count and smallest member are per-block
+// atomics, and each request's groups are the runs of constant count along its
+// row.
+//
+// Fallback (tables that break the property).  Each request computes its
+// longest common full-block prefix with every other request, sorts those
+// lengths, and reads a node's count and smallest member off the sorted list.
+// Exact for any input; O(R^2) work, used only when the check fails and
+// R <= kMaxRequestsFallback.
+//
+// Canonical order of the output: groups by (first block, smallest member);
+// members ascending.  One CTA sorts the groups in shared memory.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "fca_internal.h"
+
+namespace fca {
+namespace {
+
+
+struct RawGroup {
+    int32_t a, b, owner, nm;
+    int32_t parent_a, parent_owner, pad0, pad1;
+};
+
+struct PlanScratch {
+    int32_t* nfull;        // [R]
+    int32_t* owner;        // [NB]
+    int32_t* count;        // [NB]
+    int32_t* pos;          // [NB]
+    int32_t* valid;        // [NB] valid tokens per block (for unique bytes)
+    int32_t* n_emit;       // [R]
+    int32_t* row_goff;     // [R + 1]
+    int32_t* fill;         // [R]
+    int32_t* n_raw;        // [1]
+    RawGroup* raw;         // [R]
+    uint64_t* keys;        // [R] canonical (a << 32 | owner)
+    int32_t* g_item_off;   // [R + 1]
+    int32_t* s_item_off;   // [R + 1]
+    PlanHeader* hdr;       // [1]
+};
+
+__device__ __forceinline__ int32_t ceil_div_dev(int32_t a, int32_t b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------ validation
+
+// Thread (r, j): checks seq_lens[r] (j == 0) and table entry j if it is read.
+__global__ void k_validate(const int32_t* __restrict__ bt, int32_t MB, const int32_t* __restrict__ sl,
+                           int32_t R, int32_t NB, int32_t* __restrict__ nfull, int32_t* __restrict__ valid,
+                           PlanHeader* hdr) {
+    const int64_t total = (int64_t)R * MB;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t r = (int32_t)(i / MB), j = (int32_t)(i % MB);
+        const int32_t L = sl[r];
+        const bool len_ok = L >= 1 && (int64_t)L <= (int64_t)MB * kBlockSize;
+        if (j == 0) {
+            nfull[r] = len_ok ? L / kBlockSize : 0;
+            if (!len_ok) atomicOr(&hdr->status, kPlanBadSeqLen);
+        }
+        if (!len_ok || j >= ceil_div_dev(L, kBlockSize)) continue;
+        const int32_t b = bt[i];
+        if (b < 0 || b >= NB) {
+            atomicOr(&hdr->status, kPlanBadBlockId);
+            continue;
+        }
+        atomicMax(&valid[b], min(kBlockSize, L - j * kBlockSize));
+    }
+}
+
+// Sum of valid tokens over all blocks (each physical block once).
+__global__ void k_unique_tokens(const int32_t* __restrict__ valid, int32_t NB, PlanHeader* hdr) {
+    int64_t acc = 0;
+    for (int32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < NB; i += gridDim.x * blockDim.x) acc += valid[i];
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0 && acc) atomicAdd(reinterpret_cast<unsigned long long*>(&hdr->unique_kv_tokens),
+                                                  (unsigned long long)acc);
+}
+
+// ------------------------------------------------------------ fast path
+
+__global__ void k_block_keys(const int32_t* __restrict__ bt, int32_t MB, int32_t R,
+                             const int32_t* __restrict__ nfull, int32_t* __restrict__ owner,
+                             int32_t* __restrict__ count, int32_t* __restrict__ pos, PlanHeader* hdr) {
+    if (hdr->status & (kPlanBadSeqLen | kPlanBadBlockId)) return;
+    const int64_t total = (int64_t)R * MB;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t r = (int32_t)(i / MB), k = (int32_t)(i % MB);
+        if (k >= nfull[r]) continue;
+        const int32_t b = bt[i];
+        atomicMin(&owner[b], r);
+        atomicAdd(&count[b], 1);
+        const int32_t old = atomicCAS(&pos[b], -1, k);
+        if (old != -1 && old != k) atomicOr(&hdr->status, kPlanInconsistent);
+    }
+}
+
+__global__ void k_check_chain(const int32_t* __restrict__ bt, int32_t MB, int32_t R,
+                              const int32_t* __restrict__ nfull, const int32_t* __restrict__ owner,
+                              PlanHeader* hdr) {
+    if (hdr->status & (kPlanBadSeqLen | kPlanBadBlockId | kPlanInconsistent)) return;
+    const int64_t total = (int64_t)R * MB;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t r = (int32_t)(i / MB), k = (int32_t)(i % MB);
+        if (k == 0 || k >= nfull[r]) continue;
+        const int32_t o = owner[bt[i]];
+        if (bt[(int64_t)o * MB + k - 1] != bt[i - 1]) atomicOr(&hdr->status, kPlanInconsistent);
+    }
+}
+
+// ------------------------------------------------------------ row runs
+
+struct RowArgs {
+    const int32_t* bt;
+    int32_t MB, R, G, min_group_size, min_shared_blocks, pass;
+    const int32_t* nfull;
+    const int32_t* owner;
+    const int32_t* count;
+    PlanScratch s;
+    int32_t* suffix_start;
+    // pass 1 outputs
+    const uint64_t* keys;   // canonical keys (a << 32 | owner), n_groups of them
+    const int32_t* g_moff;
+    int32_t* members;
+    int32_t* chain_g;
+    int32_t* err;           // the plan's device error word
+};
+
+// Node information for (row, depth index k): member count and smallest member.
+struct NodeReader {
+    // fast path
+    const int32_t* row;
+    const int32_t* owner;
+    const int32_t* count;
+    // fallback: LCPs with all other requests, sorted by (lcp desc, request asc),
+    // and the running minimum of the request ids in that order
+    const int32_t* sorted_lcp;
+    const int32_t* prefix_min;
+    int32_t n_others, self;
+    bool fallback;
+
+    __device__ void at(int32_t k, int32_t& cnt, int32_t& own) const {
+        if (!fallback) {
+            const int32_t b = row[k];
+            cnt = count[b];
+            own = owner[b];
+            return;
+        }
+        // number of others whose LCP with this row exceeds k
+        int32_t lo = 0, hi = n_others;
+        while (lo < hi) {
+            const int32_t mid = (lo + hi) >> 1;
+            if (sorted_lcp[mid] > k) lo = mid + 1; else hi = mid;
+        }
+        cnt = 1 + lo;
+        own = lo > 0 ? min(self, prefix_min[lo - 1]) : self;
+    }
+};
+
+__device__ int32_t find_group(const uint64_t* keys, int32_t n, uint64_t key) {
+    int32_t lo = 0, hi = n;
+    while (lo < hi) {
+        const int32_t mid = (lo + hi) >> 1;
+        if (keys[mid] < key) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
+// One CTA per request.  Pass 0: count the request's groups, set its suffix
+// start, and (if it is a group's smallest member) record the group.  Pass 1:
+// scatter the request into its groups' member lists and its chain.
+__global__ void __launch_bounds__(256) k_row_runs(RowArgs args) {
+    extern __shared__ int32_t sm_rows[];
+    PlanHeader* hdr = args.s.hdr;
+    const int32_t status = hdr->status;
+    if (status & (kPlanBadSeqLen | kPlanBadBlockId)) return;
+    const bool fallback = (status & kPlanInconsistent) != 0;
+    if (fallback && args.R > kMaxRequestsFallback) return;
+    const int32_t R = args.R, MB = args.MB;
+    const int32_t n_groups = args.pass ? hdr->n_groups : 0;
+
+    for (int32_t r = blockIdx.x; r < R; r += gridDim.x) {
+        const int32_t nf = args.nfull[r];
+        const int32_t* row = args.bt + (int64_t)r * MB;
+        NodeReader nr;
+        nr.row = row;
+        nr.owner = args.owner;
+        nr.count = args.count;
+        nr.fallback = fallback;
+        nr.self = r;
+        nr.n_others = R - 1;
+        if (fallback) {
+            // LCP with every other request, warp-cooperative compares
+            int32_t N = 1;
+            while (N < R) N <<= 1;
+            uint64_t* key = reinterpret_cast<uint64_t*>(sm_rows);
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+            for (int32_t s = warp; s < N; s += nw) {
+                if (s >= R || s == r) {
+                    if (lane == 0) key[s] = ~0ull;
+                    continue;
+                }
+                const int32_t n = min(nf, args.nfull[s]);
+                const int32_t* other = args.bt + (int64_t)s * MB;
+                int32_t lcp = n;
+                for (int32_t base = 0; base < n; base += 32) {
+                    const int32_t k = base + lane;
+                    const bool diff = k < n && row[k] != other[k];
+                    const uint32_t m = __ballot_sync(0xffffffffu, diff);
+                    if (m) {
+                        lcp = base + __ffs(m) - 1;
+                        break;
+                    }
+                }
+                // ascending key order = lcp descending, then request ascending
+                if (lane == 0) key[s] = ((uint64_t)(uint32_t)(0x7FFFFFFF - lcp) << 32) | (uint32_t)s;
+            }
+            __syncthreads();
+            for (int32_t k = 2; k <= N; k <<= 1)
+                for (int32_t j = k >> 1; j > 0; j >>= 1) {
+                    for (int32_t i = threadIdx.x; i < N; i += blockDim.x) {
+                        const int32_t p = i ^ j;
+                        if (p > i) {
+                            const bool up = (i & k) == 0;
+                            const uint64_t x = key[i], y = key[p];
+                            if ((x > y) == up) { key[i] = y; key[p] = x; }
+                        }
+                    }
+                    __syncthreads();
+                }
+            int32_t* lcp_sorted = sm_rows + 2 * N;
+            int32_t* pmin = lcp_sorted + N;
+            if (threadIdx.x == 0) {
+                int32_t m = 0x7FFFFFFF;
+                for (int32_t i = 0; i < R - 1; ++i) {
+                    lcp_sorted[i] = 0x7FFFFFFF - (int32_t)(key[i] >> 32);
+                    m = min(m, (int32_t)(key[i] & 0xFFFFFFFFu));
+                    pmin[i] = m;
+                }
+            }
+            __syncthreads();
+            nr.sorted_lcp = lcp_sorted;
+            nr.prefix_min = pmin;
+        }
+
+        // The run scan is short and sequential in the number of runs; one
+        // thread walks the change points, the rest of the warp finds them.
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            int32_t cur_start = 0, cur_cnt = 0, cur_own = 0;
+            int32_t pending = -1, last_a = -1, last_owner = -1, last_b = 0, n_emit = 0;
+            bool done = nf == 0;
+            if (!done) {
+                nr.at(0, cur_cnt, cur_own);
+                if (cur_cnt < args.min_group_size) done = true;
+            }
+            for (int32_t base = 0; !done && base < nf; base += 32) {
+                const int32_t k = base + 1 + lane;     // candidate run end
+                int32_t c = 0, o = 0;
+                bool is_end = false;
+                if (k <= nf) {
+                    if (k == nf) {
+                        is_end = true;
+                    } else {
+                        nr.at(k, c, o);
+                        int32_t cp, op;
+                        nr.at(k - 1, cp, op);
+                        is_end = c != cp;
+                    }
+                }
+                uint32_t ends = __ballot_sync(0xffffffffu, is_end);
+                while (ends) {
+                    const int src = __ffs(ends) - 1;
+                    ends &= ends - 1;
+                    const int32_t kend = base + 1 + src;
+                    const int32_t next_c = __shfl_sync(0xffffffffu, c, src);
+                    const int32_t next_o = __shfl_sync(0xffffffffu, o, src);
+                    // close the run [cur_start, kend) with count cur_cnt
+                    const int32_t eff_a = pending >= 0 ? pending : cur_start;
+                    if (kend - eff_a < args.min_shared_blocks) {
+                        pending = eff_a;
+                    } else {
+                        if (args.pass == 0) {
+                            if (lane == 0 && cur_own == r) {
+                                const int32_t slot = atomicAdd(args.s.n_raw, 1);
+                                if (slot < R) {
+                                    RawGroup g;
+                                    g.a = eff_a;
+                                    g.b = kend;
+                                    g.owner = r;
+                                    g.nm = cur_cnt;
+                                    g.parent_a = last_a;
+                                    g.parent_owner = last_owner;
+                                    g.pad0 = g.pad1 = 0;
+                                    args.s.raw[slot] = g;
+                                } else {
+                                    atomicOr(&hdr->status, kPlanTooManyGroups);
+                                }
+                            }
+                        } else if (lane == 0) {
+                            const uint64_t key = ((uint64_t)(uint32_t)eff_a << 32) | (uint32_t)cur_own;
+                            const int32_t g = find_group(args.keys, n_groups, key);
+                            const int32_t slot = (g < n_groups && args.keys[g] == key) ? atomicAdd(&args.s.fill[g], 1)
+                                                                                     : -1;
+                            const int32_t c = args.s.row_goff[r] + n_emit;
+                            if (slot < 0 || slot >= args.g_moff[g + 1] - args.g_moff[g] || c >= args.s.row_goff[r + 1]) {
+                                atomicOr(args.err, kErrPlanInternal);   // never expected; skip the write
+                            } else {
+                                args.members[args.g_moff[g] + slot] = r;
+                                args.chain_g[c] = g;
+                            }
+                        }
+                        pending = -1;
+                        last_a = eff_a;
+                        last_owner = cur_own;
+                        last_b = kend;
+                        ++n_emit;
+                    }
+                    if (kend >= nf || next_c < args.min_group_size) {
+                        done = true;
+                        break;
+                    }
+                    cur_start = kend;
+                    cur_cnt = next_c;
+                    cur_own = next_o;
+                }
+            }
+            if (lane == 0 && args.pass == 0) {
+                args.s.n_emit[r] = n_emit;
+                args.suffix_start[r] = last_b;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------ finalize
+
+__device__ int64_t block_sum64(int64_t v, int64_t* red) {
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    int64_t t = 0;
+    if (threadIdx.x < 32) {
+        t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0;
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (threadIdx.x == 0) red[32] = t;
+    }
+    __syncthreads();
+    return red[32];
+}
+
+__device__ int32_t block_max32(int32_t v, int64_t* red) {
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        int32_t t = threadIdx.x < (blockDim.x >> 5) ? (int32_t)red[threadIdx.x] : 0;
+        for (int o = 16; o > 0; o >>= 1) t = max(t, __shfl_xor_sync(0xffffffffu, t, o));
+        if (threadIdx.x == 0) red[32] = t;
+    }
+    __syncthreads();
+    return (int32_t)red[32];
+}
+
+// Exclusive scan of f(i), i in [0, n), into out[0..n] (out[n] = total).
+// Each thread owns a contiguous run; one block-wide pass over the run sums.
+template <typename F>
+__device__ int64_t block_exclusive_scan(int32_t n, F f, int32_t* out, int64_t* red) {
+    const int32_t T = blockDim.x;
+    const int32_t per = (n + T - 1) / T;
+    const int32_t lo = min(n, (int32_t)threadIdx.x * per), hi = min(n, lo + per);
+    int64_t local = 0;
+    for (int32_t i = lo; i < hi; ++i) local += f(i);
+    // inclusive scan of per-thread sums through shared memory
+    __syncthreads();
+    red[64 + threadIdx.x] = local;
+    __syncthreads();
+    for (int32_t off = 1; off < T; off <<= 1) {
+        const int64_t v = threadIdx.x >= off ? red[64 + threadIdx.x - off] : 0;
+        __syncthreads();
+        red[64 + threadIdx.x] += v;
+        __syncthreads();
+    }
+    int64_t run = red[64 + threadIdx.x] - local;
+    const int64_t total = red[64 + T - 1];
+    for (int32_t i = lo; i < hi; ++i) {
+        out[i] = (int32_t)run;
+        run += f(i);
+    }
+    if (threadIdx.x == 0) out[n] = (int32_t)total;
+    __syncthreads();
+    return total;
+}
+
+struct FinalizeArgs {
+    PlanScratch s;
+    int32_t R, G, Hkv, split_opt, flat;
+    const int32_t* seq_lens;
+    const int32_t* suffix_start;
+    // outputs (canonical order)
+    int32_t* g_a;
+    int32_t* g_b;
+    int32_t* g_parent;
+    int32_t* g_nm;
+    int32_t* g_moff;     // [R + 1]
+    int32_t* g_nch;
+    int32_t* g_part;
+    int32_t* s_nch;
+    int32_t* s_part;
+    int32_t* chain_off;  // [R + 1]
+};
+
+// One CTA of 1024 threads.  Shared memory: sort keys (next pow2 of R, 8 B)
+// plus 64 + 1024 int64 of reduction space.
+__global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
+    extern __shared__ uint64_t sm_fin[];
+    PlanHeader* hdr = A.s.hdr;
+    if (hdr->status & (kPlanBadSeqLen | kPlanBadBlockId | kPlanTooManyGroups)) return;
+    if ((hdr->status & kPlanInconsistent) && A.R > kMaxRequestsFallback) return;
+    const int32_t R = A.R, G = A.G;
+    const int32_t n = A.flat ? 0 : min(*A.s.n_raw, R);
+    int32_t N = 1;
+    while (N < n) N <<= 1;
+    uint64_t* key = sm_fin;
+    int64_t* red = reinterpret_cast<int64_t*>(sm_fin + N);
+
+    for (int32_t i = threadIdx.x; i < N; i += blockDim.x) {
+        if (i < n) {
+            const RawGroup g = A.s.raw[i];
+            key[i] = ((uint64_t)(uint32_t)g.a << 40) | ((uint64_t)(uint32_t)g.owner << 20) | (uint32_t)i;
+        } else {
+            key[i] = ~0ull;
+        }
+    }
+    __syncthreads();
+    for (int32_t k = 2; k <= N; k <<= 1)
+        for (int32_t j = k >> 1; j > 0; j >>= 1) {
+            for (int32_t i = threadIdx.x; i < N; i += blockDim.x) {
+                const int32_t p = i ^ j;
+                if (p > i) {
+                    const bool up = (i & k) == 0;
+                    const uint64_t x = key[i], y = key[p];
+                    if ((x > y) == up) { key[i] = y; key[p] = x; }
+                }
+            }
+            __syncthreads();
+        }
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const RawGroup g = A.s.raw[key[i] & 0xFFFFF];
+        A.g_a[i] = g.a;
+        A.g_b[i] = g.b;
+        A.g_nm[i] = g.nm;
+        A.s.keys[i] = ((uint64_t)(uint32_t)g.a << 32) | (uint32_t)g.owner;
+    }
+    __syncthreads();
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const RawGroup g = A.s.raw[key[i] & 0xFFFFF];
+        int32_t par = -1;
+        if (g.parent_a >= 0) {
+            const uint64_t pk = ((uint64_t)(uint32_t)g.parent_a << 32) | (uint32_t)g.parent_owner;
+            par = find_group(A.s.keys, n, pk);
+        }
+        A.g_parent[i] = par;
+    }
+
+    // split length
+    const int32_t tile_rows = kPrefixTileRows;
+    int64_t w = 0;
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const int64_t tok = (int64_t)(A.g_b[i] - A.g_a[i]) * kBlockSize;
+        w += tok * ((A.g_nm[i] * G + tile_rows - 1) / tile_rows);
+    }
+    for (int32_t r = threadIdx.x; r < R; r += blockDim.x)
+        w += A.seq_lens[r] - (int64_t)A.suffix_start[r] * kBlockSize;
+    const int64_t work = block_sum64(w, red);
+    int32_t split = A.split_opt;
+    if (split <= 0) {
+        const int64_t target = work / 1184;   // about 8 items per SM over 148 SMs
+        split = (int32_t)std::min<int64_t>(4096, std::max<int64_t>(256, (target + 63) / 64 * 64));
+    }
+
+    // per-group chunk counts, item offsets, partial bases, member offsets
+    const int64_t n_members = block_exclusive_scan(n, [&](int32_t i) { return (int64_t)A.g_nm[i]; },
+                                                   A.g_moff, red);
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const int32_t tok = (A.g_b[i] - A.g_a[i]) * kBlockSize;
+        A.g_nch[i] = (tok + split - 1) / split;
+    }
+    __syncthreads();
+    const int64_t n_pitems = block_exclusive_scan(
+        n, [&](int32_t i) { return (int64_t)A.Hkv * A.g_nch[i] * ((A.g_nm[i] * G + tile_rows - 1) / tile_rows); },
+        A.s.g_item_off, red);
+    const int64_t n_ppart = block_exclusive_scan(
+        n, [&](int32_t i) { return (int64_t)A.Hkv * A.g_nch[i] * A.g_nm[i] * G; }, A.g_part, red);
+
+    for (int32_t r = threadIdx.x; r < R; r += blockDim.x) {
+        const int32_t tok = A.seq_lens[r] - A.suffix_start[r] * kBlockSize;
+        A.s_nch[r] = (tok + split - 1) / split;
+    }
+    __syncthreads();
+    const int64_t n_sitems = block_exclusive_scan(R, [&](int32_t r) { return (int64_t)A.Hkv * A.s_nch[r]; },
+                                                  A.s.s_item_off, red);
+    const int64_t n_spart = block_exclusive_scan(
+        R, [&](int32_t r) { return (int64_t)A.Hkv * A.s_nch[r] * G; }, A.s_part, red);
+    for (int32_t r = threadIdx.x; r < R; r += blockDim.x) A.s_part[r] += (int32_t)n_ppart;
+    const int64_t n_chain = block_exclusive_scan(
+        R, [&](int32_t r) { return A.flat ? 0 : (int64_t)A.s.n_emit[r]; }, A.chain_off, red);
+    int32_t depth = 0;
+    for (int32_t r = threadIdx.x; r < R; r += blockDim.x) depth = max(depth, A.flat ? 0 : A.s.n_emit[r]);
+    depth = block_max32(depth, red);
+
+    int64_t ptok = 0, stok = 0, ftok = 0;
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x) ptok += (int64_t)(A.g_b[i] - A.g_a[i]) * kBlockSize;
+    for (int32_t r = threadIdx.x; r < R; r += blockDim.x) {
+        stok += A.seq_lens[r] - (int64_t)A.suffix_start[r] * kBlockSize;
+        ftok += A.seq_lens[r];
+    }
+    ptok = block_sum64(ptok, red);
+    stok = block_sum64(stok, red);
+    ftok = block_sum64(ftok, red);
+    if (threadIdx.x == 0) {
+        hdr->n_groups = n;
+        hdr->n_member_entries = (int32_t)n_members;
+        hdr->max_depth = depth;
+        hdr->split_tokens = split;
+        hdr->n_prefix_items = (int32_t)n_pitems;
+        hdr->n_suffix_items = (int32_t)n_sitems;
+        hdr->n_prefix_partials = (int32_t)n_ppart;
+        hdr->n_suffix_partials = (int32_t)n_spart;
+        hdr->n_chain_entries = (int32_t)n_chain;
+        hdr->prefix_tok_sum = ptok;
+        hdr->suffix_tok_sum = stok;
+        hdr->fca_kv_tokens = ptok + stok;
+        hdr->flat_kv_tokens = ftok;
+    }
+}
+
+// One CTA per group: sort the member list, then record each member's position
+// in its chain.
+__global__ void __launch_bounds__(256) k_sort_members(const PlanHeader* hdr, const int32_t* g_moff,
+                                                      const int32_t* g_nm, int32_t* members,
+                                                      const int32_t* chain_off, const int32_t* chain_g,
+                                                      int32_t* chain_pos) {
+    extern __shared__ int32_t sm_mem[];
+    const int32_t ng = hdr->n_groups;
+    for (int32_t g = blockIdx.x; g < ng; g += gridDim.x) {
+        const int32_t off = g_moff[g], n = g_nm[g];
+        int32_t N = 1;
+        while (N < n) N <<= 1;
+        for (int32_t i = threadIdx.x; i < N; i += blockDim.x) sm_mem[i] = i < n ? members[off + i] : 0x7FFFFFFF;
+        __syncthreads();
+        for (int32_t k = 2; k <= N; k <<= 1)
+            for (int32_t j = k >> 1; j > 0; j >>= 1) {
+                for (int32_t i = threadIdx.x; i < N; i += blockDim.x) {
+                    const int32_t p = i ^ j;
+                    if (p > i) {
+                        const bool up = (i & k) == 0;
+                        const int32_t x = sm_mem[i], y = sm_mem[p];
+                        if ((x > y) == up) { sm_mem[i] = y; sm_mem[p] = x; }
+                    }
+                }
+                __syncthreads();
+            }
+        for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+            const int32_t r = sm_mem[i];
+            members[off + i] = r;
+            for (int32_t c = chain_off[r]; c < chain_off[r + 1]; ++c)
+                if (chain_g[c] == g) chain_pos[c] = i;
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------ work lists
+
+// One CTA per group: items (head, q-tile, chunk), heads outermost.
+__global__ void k_fill_prefix_items(const PlanHeader* hdr, const int32_t* g_a, const int32_t* g_b,
+                                    const int32_t* g_nm, const int32_t* g_moff, const int32_t* g_nch,
+                                    const int32_t* g_part, const int32_t* item_off, const int32_t* members,
+                                    int32_t G, int32_t Hkv, PrefixItem* items) {
+    const int32_t ng = hdr->n_groups, split = hdr->split_tokens;
+    for (int32_t g = blockIdx.x; g < ng; g += gridDim.x) {
+        const int32_t rows = g_nm[g] * G, tiles = (rows + kPrefixTileRows - 1) / kPrefixTileRows;
+        const int32_t nch = g_nch[g], per_head = tiles * nch;
+        const int32_t t0 = g_a[g] * kBlockSize, t1 = g_b[g] * kBlockSize;
+        for (int32_t i = threadIdx.x; i < Hkv * per_head; i += blockDim.x) {
+            const int32_t h = i / per_head, rem = i % per_head, tile = rem / nch, c = rem % nch;
+            PrefixItem it;
+            it.group = g;
+            it.head = h;
+            it.row0 = tile * kPrefixTileRows;
+            it.nrows = min(kPrefixTileRows, rows - it.row0);
+            it.tok0 = t0 + c * split;
+            it.tok1 = min(t1, it.tok0 + split);
+            it.bt_row = members[g_moff[g]];
+            it.part_row0 = g_part[g] + (h * nch + c) * rows + it.row0;
+            items[item_off[g] + i] = it;
+        }
+    }
+}
+
+__global__ void k_fill_suffix_items(int32_t R, const int32_t* seq_lens, const int32_t* suffix_start,
+                                    const int32_t* s_nch, const int32_t* s_part, const int32_t* item_off,
+                                    const PlanHeader* hdr, int32_t G, int32_t Hkv, SuffixItem* items) {
+    const int32_t split = hdr->split_tokens;
+    for (int32_t r = blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x) {
+        const int32_t nch = s_nch[r];
+        const int32_t t0 = suffix_start[r] * kBlockSize, L = seq_lens[r];
+        for (int32_t i = 0; i < Hkv * nch; ++i) {
+            const int32_t h = i / nch, c = i % nch;
+            SuffixItem it;
+            it.request = r;
+            it.head = h;
+            it.tok0 = t0 + c * split;
+            it.tok1 = min(L, it.tok0 + split);
+            it.part_row0 = s_part[r] + (h * nch + c) * G;
+            it.pad0 = it.pad1 = it.pad2 = 0;
+            items[item_off[r] + i] = it;
+        }
+    }
+}
+
+// ------------------------------------------------------------ host helpers
+
+// Stream-ordered temporaries, returned to the pool on scope exit.
+struct TempBuffers {
+    cudaStream_t stream;
+    std::vector<void*> ptrs;
+    bool ok = true;
+    explicit TempBuffers(cudaStream_t s) : stream(s) {}
+    ~TempBuffers() {
+        for (void* p : ptrs) cudaFreeAsync(p, stream);
+    }
+    template <typename T>
+    T* alloc(size_t count) {
+        void* p = nullptr;
+        if (cudaMallocAsync(&p, std::max<size_t>(count, 1) * sizeof(T), stream) != cudaSuccess) {
+            ok = false;
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+        ptrs.push_back(p);
+        return static_cast<T*>(p);
+    }
+};
+
+template <typename T>
+T* plan_alloc(fca_plan_s* P, size_t count, bool& ok) {
+    void* p = nullptr;
+    const size_t bytes = std::max<size_t>(count, 1) * sizeof(T);
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+        ok = false;
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    P->dev_allocs.push_back(p);
+    P->workspace_bytes += bytes;
+    return static_cast<T*>(p);
+}
+
+int grid_for(int64_t work, int threads) {
+    int64_t g = (work + threads - 1) / threads;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(g, 148 * 16));
+}
+
+int32_t next_pow2(int32_t n) {
+    int32_t N = 1;
+    while (N < n) N <<= 1;
+    return N;
+}
+
+}  // namespace
+
+#define FCA_CK(x)                                \
+    do {                                         \
+        if ((x) != cudaSuccess) {                \
+            (void)cudaGetLastError();            \
+            return FCA_ERR_CUDA;                 \
+        }                                        \
+    } while (0)
+
+// Builds the forest and work lists into P (whose shape fields are set).
+// On error the caller frees P.
+fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cudaStream_t stream,
+                      fca_plan_s* P) {
+    const int32_t R = P->R, max_blocks = P->max_blocks, num_blocks = P->num_blocks;
+    const int32_t Hkv = P->Hkv, D = P->D, G = P->G;
+    const fca_plan_opts& opts = P->opts;
+    const bool flat = P->flat;
+
+    TempBuffers tmp(stream);
+    PlanScratch s{};
+    s.nfull = tmp.alloc<int32_t>(R);
+    s.owner = tmp.alloc<int32_t>(num_blocks);
+    s.count = tmp.alloc<int32_t>(num_blocks);
+    s.pos = tmp.alloc<int32_t>(num_blocks);
+    s.valid = tmp.alloc<int32_t>(num_blocks);
+    s.n_emit = tmp.alloc<int32_t>(R);
+    s.fill = tmp.alloc<int32_t>(R);
+    s.n_raw = tmp.alloc<int32_t>(1);
+    s.raw = tmp.alloc<RawGroup>(R);
+    s.keys = tmp.alloc<uint64_t>(R);
+    s.g_item_off = tmp.alloc<int32_t>(R + 1);
+    s.s_item_off = tmp.alloc<int32_t>(R + 1);
+    s.hdr = tmp.alloc<PlanHeader>(1);
+    bool ok = tmp.ok;
+    P->bt = plan_alloc<int32_t>(P, (size_t)R * max_blocks, ok);
+    P->seq_lens = plan_alloc<int32_t>(P, R, ok);
+    P->suffix_start = plan_alloc<int32_t>(P, R, ok);
+    P->g_a = plan_alloc<int32_t>(P, R, ok);
+    P->g_b = plan_alloc<int32_t>(P, R, ok);
+    P->g_parent = plan_alloc<int32_t>(P, R, ok);
+    P->g_nm = plan_alloc<int32_t>(P, R, ok);
+    P->g_moff = plan_alloc<int32_t>(P, R + 1, ok);
+    P->g_nch = plan_alloc<int32_t>(P, R, ok);
+    P->g_part = plan_alloc<int32_t>(P, R + 1, ok);
+    P->s_nch = plan_alloc<int32_t>(P, R, ok);
+    P->s_part = plan_alloc<int32_t>(P, R + 1, ok);
+    P->chain_off = plan_alloc<int32_t>(P, R + 1, ok);
+    P->dev_status = plan_alloc<int32_t>(P, 1, ok);
+    if (!ok) return FCA_ERR_OOM;
+    s.row_goff = P->chain_off;
+
+    FCA_CK(cudaMemcpyAsync(P->bt, block_tables, sizeof(int32_t) * (size_t)R * max_blocks,
+                           cudaMemcpyDeviceToDevice, stream));
+    FCA_CK(cudaMemcpyAsync(P->seq_lens, seq_lens, sizeof(int32_t) * R, cudaMemcpyDeviceToDevice, stream));
+    FCA_CK(cudaMemsetAsync(s.owner, 0x7F, sizeof(int32_t) * (size_t)num_blocks, stream));
+    FCA_CK(cudaMemsetAsync(s.count, 0, sizeof(int32_t) * (size_t)num_blocks, stream));
+    FCA_CK(cudaMemsetAsync(s.pos, 0xFF, sizeof(int32_t) * (size_t)num_blocks, stream));
+    FCA_CK(cudaMemsetAsync(s.valid, 0, sizeof(int32_t) * (size_t)num_blocks, stream));
+    FCA_CK(cudaMemsetAsync(s.n_raw, 0, sizeof(int32_t), stream));
+    FCA_CK(cudaMemsetAsync(s.fill, 0, sizeof(int32_t) * R, stream));
+    FCA_CK(cudaMemsetAsync(s.n_emit, 0, sizeof(int32_t) * R, stream));
+    FCA_CK(cudaMemsetAsync(s.hdr, 0, sizeof(PlanHeader), stream));
+    FCA_CK(cudaMemsetAsync(P->suffix_start, 0, sizeof(int32_t) * R, stream));
+    FCA_CK(cudaMemsetAsync(P->dev_status, 0, sizeof(int32_t), stream));
+
+    const int64_t cells = (int64_t)R * max_blocks;
+    k_validate<<<grid_for(cells, 256), 256, 0, stream>>>(P->bt, max_blocks, P->seq_lens, R, num_blocks, s.nfull,
+                                                         s.valid, s.hdr);
+    k_unique_tokens<<<grid_for(num_blocks, 256), 256, 0, stream>>>(s.valid, num_blocks, s.hdr);
+    FCA_CK(cudaGetLastError());
+
+    RowArgs ra{};
+    size_t row_smem = 0;
+    const int row_grid = std::min(R, 148 * 8);
+    if (!flat) {
+        k_block_keys<<<grid_for(cells, 256), 256, 0, stream>>>(P->bt, max_blocks, R, s.nfull, s.owner, s.count,
+                                                               s.pos, s.hdr);
+        k_check_chain<<<grid_for(cells, 256), 256, 0, stream>>>(P->bt, max_blocks, R, s.nfull, s.owner, s.hdr);
+        ra.bt = P->bt;
+        ra.MB = max_blocks;
+        ra.R = R;
+        ra.G = G;
+        ra.min_group_size = opts.min_group_size;
+        ra.min_shared_blocks = opts.min_shared_blocks;
+        ra.pass = 0;
+        ra.nfull = s.nfull;
+        ra.owner = s.owner;
+        ra.count = s.count;
+        ra.s = s;
+        ra.suffix_start = P->suffix_start;
+        // the fallback keeps 8-byte sort keys and two int32 arrays per request
+        row_smem = R <= kMaxRequestsFallback ? (size_t)next_pow2(R) * 16 : 0;
+        FCA_CK(cudaFuncSetAttribute(k_row_runs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)row_smem));
+        k_row_runs<<<row_grid, 256, row_smem, stream>>>(ra);
+        FCA_CK(cudaGetLastError());
+    }
+
+    FinalizeArgs fa{};
+    fa.s = s;
+    fa.R = R;
+    fa.G = G;
+    fa.Hkv = Hkv;
+    fa.split_opt = opts.split_tokens;
+    fa.flat = flat ? 1 : 0;
+    fa.seq_lens = P->seq_lens;
+    fa.suffix_start = P->suffix_start;
+    fa.g_a = P->g_a;
+    fa.g_b = P->g_b;
+    fa.g_parent = P->g_parent;
+    fa.g_nm = P->g_nm;
+    fa.g_moff = P->g_moff;
+    fa.g_nch = P->g_nch;
+    fa.g_part = P->g_part;
+    fa.s_nch = P->s_nch;
+    fa.s_part = P->s_part;
+    fa.chain_off = P->chain_off;
+    const size_t fin_smem = (size_t)next_pow2(R) * 8 + (64 + 1024) * 8;
+    FCA_CK(cudaFuncSetAttribute(k_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem));
+    k_finalize<<<1, 1024, fin_smem, stream>>>(fa);
+    FCA_CK(cudaGetLastError());
+
+    // the one synchronisation: sizes of the forest and of the work lists
+    FCA_CK(cudaMemcpyAsync(&P->hdr, s.hdr, sizeof(PlanHeader), cudaMemcpyDeviceToHost, stream));
+    FCA_CK(cudaStreamSynchronize(stream));
+    const PlanHeader& H = P->hdr;
+    if (H.status & kPlanBadSeqLen) return FCA_ERR_INVALID_ARG;
+    if (H.status & kPlanBadBlockId) return FCA_ERR_BAD_BLOCK_ID;
+    if (H.status & kPlanTooManyGroups) return FCA_ERR_UNSUPPORTED;
+    if ((H.status & kPlanInconsistent) && R > kMaxRequestsFallback) return FCA_ERR_UNSUPPORTED;
+    const int64_t n_part = (int64_t)H.n_prefix_partials + H.n_suffix_partials;
+    if (n_part >= (int64_t)INT32_MAX / 2) return FCA_ERR_UNSUPPORTED;
+
+    P->members = plan_alloc<int32_t>(P, H.n_member_entries, ok);
+    P->chain_g = plan_alloc<int32_t>(P, H.n_chain_entries, ok);
+    P->chain_pos = plan_alloc<int32_t>(P, H.n_chain_entries, ok);
+    P->prefix_items = plan_alloc<PrefixItem>(P, H.n_prefix_items, ok);
+    P->suffix_items = plan_alloc<SuffixItem>(P, H.n_suffix_items, ok);
+    P->part_o = plan_alloc<float>(P, (size_t)n_part * D, ok);
+    P->part_lse = plan_alloc<float>(P, n_part, ok);
+    if (!ok) return FCA_ERR_OOM;
+
+    if (!flat && H.n_groups > 0) {
+        ra.pass = 1;
+        ra.keys = s.keys;
+        ra.g_moff = P->g_moff;
+        ra.members = P->members;
+        ra.chain_g = P->chain_g;
+        ra.err = P->dev_status;
+        k_row_runs<<<row_grid, 256, row_smem, stream>>>(ra);
+        FCA_CK(cudaGetLastError());
+        const size_t mem_smem = (size_t)next_pow2(R) * 4;
+        FCA_CK(cudaFuncSetAttribute(k_sort_members, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mem_smem));
+        k_sort_members<<<std::min(H.n_groups, 148 * 4), 256, mem_smem, stream>>>(
+            s.hdr, P->g_moff, P->g_nm, P->members, P->chain_off, P->chain_g, P->chain_pos);
+        k_fill_prefix_items<<<std::min(H.n_groups, 148 * 4), 256, 0, stream>>>(
+            s.hdr, P->g_a, P->g_b, P->g_nm, P->g_moff, P->g_nch, P->g_part, s.g_item_off, P->members, G, Hkv,
+            P->prefix_items);
+        FCA_CK(cudaGetLastError());
+    }
+    if (H.n_suffix_items > 0) {
+        k_fill_suffix_items<<<grid_for(R, 128), 128, 0, stream>>>(R, P->seq_lens, P->suffix_start, P->s_nch,
+                                                                  P->s_part, s.s_item_off, s.hdr, G, Hkv,
+                                                                  P->suffix_items);
+        FCA_CK(cudaGetLastError());
+    }
+    return FCA_OK;   // temporaries go back to the pool in stream order
+}
+
+#undef FCA_CK
+
+}  // namespace fca

@@ -1,0 +1,84 @@
+"""The C-ABI library loads and exports everything include/fca.h declares.
+
+No GPU needed: only calls that return before touching the device are made
+(status strings, version, default options, argument checks).
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import shared_prefix_kv_fca_b200 as fca
+from shared_prefix_kv_fca_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "fca.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(fca_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fbuild.build()
+    return fca.load_library()
+
+
+def test_header_declares_the_expected_entry_points():
+    names = declared_functions()
+    for n in ["fca_plan", "fca_decode", "fca_flat_decode", "fca_plan_get_stats", "fca_plan_export",
+              "fca_plan_member_count", "fca_plan_destroy", "fca_check_device_status",
+              "fca_status_string", "fca_version", "fca_plan_opts_default"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", fca.library_path()]).decode()
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_library_is_built_for_sm100a_only():
+    assert fbuild.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_host_only_calls(lib):
+    assert fca.fca_version().startswith("fca_b200")
+    assert fca.fca_status_string(0) == "ok"
+    assert fca.fca_status_string(2) == "block id out of range"
+    o = fca.fca_plan_opts_default()
+    assert (o.min_group_size, o.min_shared_blocks, o.split_tokens, o.flags) == (2, 1, 0, 0)
+
+
+def test_argument_checks_return_status_without_a_device(lib):
+    h = ctypes.c_void_p()
+    opts = fca.fca_plan_opts_default()
+    fake = ctypes.c_void_p(16)  # never dereferenced: every call below fails its host checks
+    # no output handle
+    assert lib.fca_plan(fake, 4, fake, 2, 16, 8, 4, 1, 64, ctypes.byref(opts), None, None) == 1
+    # null tables
+    assert lib.fca_plan(None, 4, fake, 2, 16, 8, 4, 1, 64, ctypes.byref(opts), ctypes.byref(h), None) == 1
+    # Hq not a multiple of Hkv
+    assert lib.fca_plan(fake, 4, fake, 2, 16, 8, 6, 4, 64, ctypes.byref(opts), ctypes.byref(h), None) == 1
+    # head_dim / block_size not built
+    assert lib.fca_plan(fake, 4, fake, 2, 16, 8, 4, 1, 96, ctypes.byref(opts), ctypes.byref(h), None) == 3
+    assert lib.fca_plan(fake, 4, fake, 2, 32, 8, 4, 1, 64, ctypes.byref(opts), ctypes.byref(h), None) == 3
+    # GQA ratio above the built maximum
+    assert lib.fca_plan(fake, 4, fake, 2, 16, 8, 32, 1, 64, ctypes.byref(opts), ctypes.byref(h), None) == 3
+    # bad options
+    bad = fca.fca_plan_opts(1, 1, 0, 0)
+    assert lib.fca_plan(fake, 4, fake, 2, 16, 8, 4, 1, 64, ctypes.byref(bad), ctypes.byref(h), None) == 1
+    bad = fca.fca_plan_opts(2, 1, 100, 0)
+    assert lib.fca_plan(fake, 4, fake, 2, 16, 8, 4, 1, 64, ctypes.byref(bad), ctypes.byref(h), None) == 1
+    assert h.value is None
+    # decode without a plan, flat decode without a plan
+    assert lib.fca_decode(fake, fake, fake, None, fake, None, 0.1, None) == 1
+    assert lib.fca_flat_decode(fake, fake, fake, None, fake, None, 0.1, None) == 1
+    assert lib.fca_plan_destroy(None) == 0

@@ -1,0 +1,236 @@
+"""CUDA path vs the CPU oracle, through the C ABI.
+
+Plans must match the oracle planner bit for bit.  Attention outputs (bf16
+inputs, fp32 accumulation, bf16 output) must be within max-abs 1e-2 and
+mean-abs 1e-3 of the oracle's fp64 result, and the LSE within 1e-3
+(absolute, natural log).  Small cases compare every output; the full-size
+configurations compare sampled (request, head) pairs against the oracle and
+every output against the flat paged decode kernel.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import fca_workloads
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+TOL_MAX, TOL_MEAN, TOL_LSE = 1e-2, 1e-3, 1e-3
+
+
+def _torch():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch
+
+
+def run(w, flat=False, lse=True, **opts):
+    """Plan + decode through the binding; returns (out f64 [R,Hq,D], lse f64, plan export, stats)."""
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    q, k, v, bt, sl = w.torch_inputs("cuda")
+    plan = fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, flat=flat, **opts)
+    out = torch.empty_like(q)
+    l = torch.empty(w.R, w.Hq, dtype=torch.float32, device="cuda") if lse else None
+    (fca.fca_flat_decode if flat else fca.fca_decode)(q, k, v, plan, out, l, w.scale)
+    assert fca.fca_check_device_status(plan) == 0
+    exp = plan.export()
+    st = plan.stats()
+    plan.close()
+    o = out.float().cpu().numpy().astype(np.float64)
+    return o, (l.cpu().numpy().astype(np.float64) if lse else None), exp, st
+
+
+def assert_close(o, l, o_ref, l_ref, what=""):
+    err = np.abs(o - o_ref)
+    assert np.isfinite(o).all(), f"{what}: non-finite output"
+    assert err.max() <= TOL_MAX, f"{what}: max-abs {err.max():.3e}"
+    assert err.mean() <= TOL_MEAN, f"{what}: mean-abs {err.mean():.3e}"
+    if l is not None:
+        le = np.abs(l - l_ref).max()
+        assert le <= TOL_LSE, f"{what}: lse err {le:.3e}"
+
+
+def assert_plan_equal(exp, ref):
+    for key in ("a", "b", "parent", "member_off", "n_members", "members", "suffix_start"):
+        np.testing.assert_array_equal(exp[key], ref[key], err_msg=key)
+
+
+# --------------------------------------------------------------- planner
+
+@pytest.mark.parametrize("seed", range(30))
+def test_plan_bit_exact_random_forests(seed):
+    w = fca_workloads.random_small(seed, max_requests=24)
+    _, _, exp, st = run(w)
+    assert_plan_equal(exp, oracle.plan(w.block_tables, w.seq_lens, w.block_size))
+    assert st["unique_kv_tokens"] == oracle.unique_kv_tokens(w.block_tables, w.seq_lens,
+                                                               w.block_size, w.num_blocks)
+
+
+@pytest.mark.parametrize("mgs,msb", [(3, 1), (2, 2), (4, 3), (2, 5)])
+def test_plan_options(mgs, msb):
+    for seed in range(12):
+        w = fca_workloads.random_small(seed, max_requests=24)
+        _, _, exp, _ = run(w, min_group_size=mgs, min_shared_blocks=msb)
+        assert_plan_equal(exp, oracle.plan(w.block_tables, w.seq_lens, w.block_size, mgs, msb))
+
+
+def inconsistent_workload():
+    """Tables whose block ids do not identify prefixes: block 11 sits under two
+    different parents, block 20 at two logical positions."""
+    w = fca_workloads.random_small(2, Hq=4, Hkv=2, D=64)
+    B = 16
+    bt = np.array([[10, 11, 12, 13, 30],
+                   [10, 11, 12, 14, 31],
+                   [15, 11, 12, 13, 32],
+                   [15, 11, 12, 13, 33],
+                   [20, 21, 22, 34, 0],
+                   [23, 20, 21, 35, 0],
+                   [10, 11, 16, 36, 37]], np.int32)
+    sl = np.array([5 * B - 3, 5 * B, 4 * B + 1, 4 * B + 9, 3 * B + 2, 4 * B, 5 * B - 1], np.int32)
+    nb = 40
+    k = fca_workloads.normal_bf16((nb, B, w.Hkv, w.D), 5, 1)
+    v = fca_workloads.normal_bf16((nb, B, w.Hkv, w.D), 5, 2)
+    q = fca_workloads.normal_bf16((bt.shape[0], w.Hq, w.D), 5, 0)
+    return fca_workloads.Workload("inconsistent", q, k, v, bt, sl, w.Hq, w.Hkv, w.D, B, 5)
+
+
+def test_plan_fallback_for_tables_without_prefix_identity():
+    w = inconsistent_workload()
+    o, l, exp, _ = run(w)
+    ref = oracle.plan(w.block_tables, w.seq_lens, w.block_size)
+    assert_plan_equal(exp, ref)
+    assert len(ref["a"]) >= 3
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(o, l, o_ref, l_ref, "fallback plan decode")
+
+
+def test_plan_named_configs_bit_exact():
+    for name in ("tiny", "llama8b", "forest", "longctx"):
+        w = fca_workloads.make(name)
+        torch = _torch()
+        import shared_prefix_kv_fca_b200 as fca
+        bt = torch.from_numpy(w.block_tables).cuda()
+        sl = torch.from_numpy(w.seq_lens).cuda()
+        with fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D) as plan:
+            exp = plan.export()
+            st = plan.stats()
+        assert_plan_equal(exp, oracle.plan(w.block_tables, w.seq_lens, 16))
+        assert st["unique_kv_tokens"] == oracle.unique_kv_tokens(w.block_tables, w.seq_lens, 16,
+                                                                   w.num_blocks)
+
+
+# --------------------------------------------------------------- attention, all outputs
+
+@pytest.mark.parametrize("seed", range(12))
+@pytest.mark.parametrize("flat", [False, True])
+def test_decode_matches_oracle_random(seed, flat):
+    Hq, Hkv, D = [(4, 2, 64), (8, 2, 128), (4, 4, 128), (16, 2, 64), (6, 2, 128), (8, 1, 128)][seed % 6]
+    w = fca_workloads.random_small(seed, Hq=Hq, Hkv=Hkv, D=D, max_requests=20,
+                                   poison_padding=seed % 2 == 1)
+    o, l, _, _ = run(w, flat=flat)
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(o, l, o_ref, l_ref, f"seed {seed} flat={flat}")
+
+
+@pytest.mark.parametrize("split", [64, 128, 256])
+def test_decode_small_splits(split):
+    # many split chunks per group and per request, ragged tails
+    for seed in (3, 7):
+        w = fca_workloads.random_small(seed, Hq=8, Hkv=2, D=128, max_requests=16)
+        o, l, _, _ = run(w, split_tokens=split)
+        o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens,
+                                              w.scale)
+        assert_close(o, l, o_ref, l_ref, f"split {split}")
+
+
+def test_tiny_config_all_outputs():
+    w = fca_workloads.make("tiny", poison_padding=True)
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    for flat in (False, True):
+        o, l, _, _ = run(w, flat=flat)
+        assert_close(o, l, o_ref, l_ref, f"tiny flat={flat}")
+
+
+def test_lse_optional():
+    w = fca_workloads.random_small(4, D=64)
+    o, l, _, _ = run(w, lse=False)
+    o_ref, _ = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(o, None, o_ref, None, "no lse")
+
+
+# --------------------------------------------------------------- full-size configurations
+
+def sampled_pairs(w, n, seed=0):
+    rng = np.random.default_rng(seed)
+    r = rng.integers(0, w.R, size=n)
+    h = rng.integers(0, w.Hq, size=n)
+    # always include the longest and shortest request
+    r[0], r[1] = int(np.argmax(w.seq_lens)), int(np.argmin(w.seq_lens))
+    return np.stack([r, h], 1).astype(np.int32)
+
+
+@pytest.mark.parametrize("name", ["llama8b", "longctx", "forest", "mixed"])
+def test_full_size_configs(name):
+    w = fca_workloads.make(name)
+    o, l, exp, st = run(w)
+    of, lf, _, _ = run(w, flat=True)
+    pairs = sampled_pairs(w, 128)
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens,
+                                          w.scale, pairs=pairs)
+    sel = (pairs[:, 0], pairs[:, 1])
+    assert_close(o[sel], l[sel], o_ref, l_ref, f"{name} fca sampled")
+    assert_close(of[sel], lf[sel], o_ref, l_ref, f"{name} flat sampled")
+    # every output: FCA equals the flat (standard) attention kernel.  Both are
+    # within the oracle tolerance of the exact result, so they are within twice
+    # that of each other (one bf16 ulp is already 1.56e-2 for |o| in [2, 4)).
+    err = np.abs(o - of)
+    assert np.isfinite(o).all() and np.isfinite(of).all()
+    assert err.max() <= 2 * TOL_MAX, f"{name} fca vs flat: max-abs {err.max():.3e}"
+    assert err.mean() <= 2 * TOL_MEAN, f"{name} fca vs flat: mean-abs {err.mean():.3e}"
+    assert np.abs(l - lf).max() <= 2 * TOL_LSE
+    assert st["unique_kv_bytes"] == oracle.unique_kv_tokens(
+        w.block_tables, w.seq_lens, 16, w.num_blocks) * w.Hkv * w.D * 4
+
+
+# --------------------------------------------------------------- errors
+
+def test_error_paths_return_status():
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    w = fca_workloads.random_small(1, D=64)
+    bt = torch.from_numpy(w.block_tables).cuda()
+    sl = torch.from_numpy(w.seq_lens).cuda()
+    bad = w.block_tables.copy()
+    bad[0, 0] = w.num_blocks + 5
+    with pytest.raises(fca.FcaError) as e:
+        fca.fca_plan(torch.from_numpy(bad).cuda(), sl, w.num_blocks, w.Hq, w.Hkv, w.D)
+    assert e.value.status == 2
+    bad = w.block_tables.copy()
+    bad[0, 0] = -1
+    with pytest.raises(fca.FcaError) as e:
+        fca.fca_plan(torch.from_numpy(bad).cuda(), sl, w.num_blocks, w.Hq, w.Hkv, w.D)
+    assert e.value.status == 2
+    for L in (0, w.max_blocks * 16 + 1):
+        s2 = w.seq_lens.copy()
+        s2[-1] = L
+        with pytest.raises(fca.FcaError) as e:
+            fca.fca_plan(bt, torch.from_numpy(s2).cuda(), w.num_blocks, w.Hq, w.Hkv, w.D)
+        assert e.value.status == 1
+    with pytest.raises(fca.FcaError) as e:
+        fca.fca_plan(bt, sl, w.num_blocks, 6, 4, w.D)
+    assert e.value.status == 1
+    with pytest.raises(fca.FcaError) as e:
+        fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, 96)
+    assert e.value.status == 3
+    # a flat decode needs a flat plan
+    q, k, v, _, _ = w.torch_inputs("cuda")
+    with fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D) as plan:
+        with pytest.raises(fca.FcaError):
+            fca.fca_flat_decode(q, k, v, plan, torch.empty_like(q))
+        # the good plan still works after the failed calls
+        out = torch.empty_like(q)
+        fca.fca_decode(q, k, v, plan, out)
+        assert fca.fca_check_device_status(plan) == 0
