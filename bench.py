@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--impl", choices=["fca", "reference"], default="fca")
     ap.add_argument("--config", default="llama8b")
     ap.add_argument("--split", type=int, default=0, help="split-KV chunk tokens (0 = automatic)")
+    ap.add_argument("--prompts", type=int, default=None,
+                    help="shrink the configuration to this many prompts (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-flat", action="store_true")
@@ -189,7 +191,7 @@ def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = fca_workloads.make(args.config, seed=0)
+    w = fca_workloads.make(args.config, seed=0, prompts=args.prompts)
     ub = unique_bytes(w)
     total_tok = int(w.seq_lens.sum())
     per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
@@ -267,7 +269,7 @@ def fca_arm(args):
         dist.all_reduce(t, op=dist.ReduceOp.SUM)
         return float(t.item())
 
-    w = fca_workloads.make(args.config, seed=rank)
+    w = fca_workloads.make(args.config, seed=rank, prompts=args.prompts)
     q, k, v, bt, sl = w.torch_inputs(dev)
     stream = torch.cuda.current_stream(dev)
     out = torch.empty_like(q)

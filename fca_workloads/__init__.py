@@ -256,8 +256,11 @@ def _zipf_truncated(rng, s: float, kmax: int, total: int):
     return sizes
 
 
-def make(name: str, seed: int = 0, poison_padding: bool = False) -> Workload:
-    """One of the named configurations (see module docstring)."""
+def make(name: str, seed: int = 0, poison_padding: bool = False,
+         prompts: Optional[int] = None) -> Workload:
+    """One of the named configurations (see module docstring).  ``prompts``
+    shrinks ``llama8b`` / ``longctx`` / ``forest`` to that many prompts (same
+    per-prompt structure), for profiling captures that must stay small."""
     rng = np.random.default_rng(seed)
     c = CONFIGS[name]
     reqs = []
@@ -269,21 +272,21 @@ def make(name: str, seed: int = 0, poison_padding: bool = False) -> Workload:
         return fill(name, reqs, seed=seed, rng=rng, poison_padding=poison_padding,
                     description=desc, **c)
     if name == "llama8b":
-        for p in range(16):
+        for p in range(prompts or 16):
             for _ in range(16):
                 reqs.append([(f"p{p}", 2048), (None, int(rng.integers(1, 1025)))])
         desc = "16 prompts x 16 samples, prompt 2048 tokens, own U{1..1024}"
         return fill(name, reqs, seed=seed, rng=rng, poison_padding=poison_padding,
                     description=desc, **c)
     if name == "longctx":
-        for p in range(4):
+        for p in range(prompts or 4):
             for _ in range(16):
                 reqs.append([(f"p{p}", 32768), (None, int(rng.integers(1, 8193)))])
         desc = "4 prompts x 16 samples, prompt 32768 tokens, own U{1..8192}, K x3 on 1% of slots"
         return fill(name, reqs, seed=seed, rng=rng, k_boost_frac=0.01,
                     poison_padding=poison_padding, description=desc, **c)
     if name == "forest":
-        for p in range(32):
+        for p in range(prompts or 32):
             for _ in range(16):
                 reqs.append([("sys", 1024), (f"p{p}", 2048), (None, int(rng.integers(0, 513)))])
         desc = "512 requests: 1024-token system prompt, 32 prompts x 2048 tokens x 16 samples, own U{0..512}"

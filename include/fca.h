@@ -147,7 +147,8 @@ fca_status fca_merge_pass(fca_plan_t plan, void *out, float *lse, void *stream);
 /* Sizes and byte counts of a plan (HOST struct, filled synchronously). */
 typedef struct fca_plan_stats {
     int32_t num_requests, num_groups, max_depth, num_q_heads, num_kv_heads, head_dim;
-    int32_t split_tokens;           /* chunk length actually used */
+    int32_t split_tokens;           /* chunk target of the per-request pass */
+    int32_t prefix_split_tokens;    /* chunk target of the grouped pass */
     int32_t prefix_items, suffix_items;   /* work items of the two passes */
     int64_t num_partials;           /* partial (o, lse) rows written per decode */
     int64_t unique_kv_tokens;       /* each referenced physical block once, its valid tokens */
@@ -190,6 +191,10 @@ fca_status fca_plan_destroy(fca_plan_t plan);
  * word was non-zero.
  */
 fca_status fca_check_device_status(fca_plan_t plan, void *stream, int32_t *code);
+
+/* Text of the last CUDA error a call of this library met on the calling
+ * thread ("no error" if none); valid until the next failing call. */
+const char *fca_last_cuda_error(void);
 
 /* Static description of a status code. */
 const char *fca_status_string(fca_status status);

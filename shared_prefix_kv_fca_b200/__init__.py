@@ -26,7 +26,7 @@ __all__ = [
     "FcaError", "Plan", "fca_plan", "fca_decode", "fca_flat_decode", "fca_plan_get_stats",
     "fca_plan_export", "fca_plan_member_count", "fca_plan_destroy", "fca_check_device_status",
     "fca_status_string", "fca_version", "fca_plan_opts_default", "library_path", "load_library",
-    "fca_prefix_pass", "fca_suffix_pass", "fca_merge_pass",
+    "fca_prefix_pass", "fca_suffix_pass", "fca_merge_pass", "fca_last_cuda_error",
     "FCA_PLAN_FLAT", "STATUS",
 ]
 
@@ -42,7 +42,10 @@ STATUS = {0: "FCA_OK", 1: "FCA_ERR_INVALID_ARG", 2: "FCA_ERR_BAD_BLOCK_ID", 3: "
 class FcaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS.get(status, status)} ({fca_status_string(status)})")
+        msg = f"{where}: {STATUS.get(status, status)} ({fca_status_string(status)})"
+        if status == 4:
+            msg += f": {load_library().fca_last_cuda_error().decode()}"
+        super().__init__(msg)
 
 
 class fca_plan_opts(ctypes.Structure):
@@ -54,7 +57,8 @@ class fca_plan_stats(ctypes.Structure):
     _fields_ = [("num_requests", ctypes.c_int32), ("num_groups", ctypes.c_int32),
                 ("max_depth", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("split_tokens", ctypes.c_int32), ("prefix_items", ctypes.c_int32),
+                ("split_tokens", ctypes.c_int32), ("prefix_split_tokens", ctypes.c_int32),
+                ("prefix_items", ctypes.c_int32),
                 ("suffix_items", ctypes.c_int32), ("num_partials", ctypes.c_int64),
                 ("unique_kv_tokens", ctypes.c_int64), ("unique_kv_bytes", ctypes.c_int64),
                 ("flat_kv_bytes", ctypes.c_int64), ("fca_kv_bytes", ctypes.c_int64),
@@ -106,6 +110,8 @@ def load_library():
     lib.fca_status_string.restype = ctypes.c_char_p
     lib.fca_version.argtypes = []
     lib.fca_version.restype = ctypes.c_char_p
+    lib.fca_last_cuda_error.argtypes = []
+    lib.fca_last_cuda_error.restype = ctypes.c_char_p
     _lib = lib
     return lib
 
@@ -134,6 +140,10 @@ def fca_status_string(status: int) -> str:
 
 def fca_version() -> str:
     return load_library().fca_version().decode()
+
+
+def fca_last_cuda_error() -> str:
+    return load_library().fca_last_cuda_error().decode()
 
 
 def fca_plan_opts_default() -> fca_plan_opts:

@@ -9,11 +9,20 @@
 
 namespace fca {
 fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cudaStream_t stream, fca_plan_s* P);
-cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
-                          float scale, cudaStream_t stream);
+cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const void* k_cache, const void* v_cache,
+                          const CUtensorMap& tk, const CUtensorMap& tv, float scale, cudaStream_t stream);
 cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
                           float scale, cudaStream_t stream);
 cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, cudaStream_t stream);
+
+namespace {
+thread_local cudaError_t g_last_error = cudaSuccess;
+}  // namespace
+
+cudaError_t note_cuda(cudaError_t e) {
+    if (e != cudaSuccess) g_last_error = e;
+    return e;
+}
 
 namespace {
 
@@ -126,10 +135,10 @@ static fca_status decode_impl(const void* q, const void* k_cache, const void* v_
     if (!make_cache_map(&tk, k_cache, plan->num_blocks, plan->Hkv, plan->D) ||
         !make_cache_map(&tv, v_cache, plan->num_blocks, plan->Hkv, plan->D))
         return FCA_ERR_CUDA;
-    if (!plan->flat && plan->hdr.n_prefix_items > 0 && launch_prefix(plan, q, tk, tv, scale, s) != cudaSuccess)
+    if (!plan->flat && plan->hdr.n_prefix_items > 0 && note_cuda(launch_prefix(plan, q, k_cache, v_cache, tk, tv, scale, s)) != cudaSuccess)
         return FCA_ERR_CUDA;
-    if (launch_suffix(plan, q, tk, tv, scale, s) != cudaSuccess) return FCA_ERR_CUDA;
-    if (launch_merge(plan, out, lse, s) != cudaSuccess) return FCA_ERR_CUDA;
+    if (note_cuda(launch_suffix(plan, q, tk, tv, scale, s)) != cudaSuccess) return FCA_ERR_CUDA;
+    if (note_cuda(launch_merge(plan, out, lse, s)) != cudaSuccess) return FCA_ERR_CUDA;
     return FCA_OK;
 }
 
@@ -149,9 +158,9 @@ static fca_status pass_impl(int pass, const void* q, const void* k_cache, const 
         return FCA_ERR_CUDA;
     if (pass == 0) {
         if (plan->flat || plan->hdr.n_prefix_items == 0) return FCA_OK;
-        return launch_prefix(plan, q, tk, tv, scale, s) == cudaSuccess ? FCA_OK : FCA_ERR_CUDA;
+        return note_cuda(launch_prefix(plan, q, k_cache, v_cache, tk, tv, scale, s)) == cudaSuccess ? FCA_OK : FCA_ERR_CUDA;
     }
-    return launch_suffix(plan, q, tk, tv, scale, s) == cudaSuccess ? FCA_OK : FCA_ERR_CUDA;
+    return note_cuda(launch_suffix(plan, q, tk, tv, scale, s)) == cudaSuccess ? FCA_OK : FCA_ERR_CUDA;
 }
 
 fca_status fca_prefix_pass(const void* q, const void* k_cache, const void* v_cache, fca_plan_t plan, float scale,
@@ -167,8 +176,9 @@ fca_status fca_suffix_pass(const void* q, const void* k_cache, const void* v_cac
 fca_status fca_merge_pass(fca_plan_t plan, void* out, float* lse, void* stream) {
     if (!plan || !out || !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return FCA_ERR_INVALID_ARG;
-    return launch_merge(plan, out, lse, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FCA_OK
-                                                                                          : FCA_ERR_CUDA;
+    return note_cuda(launch_merge(plan, out, lse, static_cast<cudaStream_t>(stream))) == cudaSuccess
+               ? FCA_OK
+               : FCA_ERR_CUDA;
 }
 
 fca_status fca_flat_decode(const void* q, const void* k_cache, const void* v_cache, fca_plan_t plan, void* out,
@@ -188,6 +198,7 @@ fca_status fca_plan_get_stats(fca_plan_t plan, fca_plan_stats* st) {
     st->num_kv_heads = plan->Hkv;
     st->head_dim = plan->D;
     st->split_tokens = H.split_tokens;
+    st->prefix_split_tokens = H.prefix_split_tokens;
     st->prefix_items = H.n_prefix_items;
     st->suffix_items = H.n_suffix_items;
     st->num_partials = (int64_t)H.n_prefix_partials + H.n_suffix_partials;
@@ -264,5 +275,7 @@ const char* fca_status_string(fca_status status) {
 }
 
 const char* fca_version(void) { return "fca_b200 0.1.0 sm_100a"; }
+
+const char* fca_last_cuda_error(void) { return cudaGetErrorString(g_last_error); }
 
 }  // extern "C"

@@ -52,7 +52,8 @@ struct PlanHeader {
     int32_t n_groups;
     int32_t n_member_entries;   // sum of group sizes
     int32_t max_depth;
-    int32_t split_tokens;
+    int32_t split_tokens;       // chunk target of the per-request pass
+    int32_t prefix_split_tokens;// chunk target of the grouped pass
     int32_t n_prefix_items;
     int32_t n_suffix_items;
     int32_t n_prefix_partials;  // partial rows written by the grouped pass
@@ -64,6 +65,9 @@ struct PlanHeader {
     int64_t prefix_tok_sum;     // sum over groups of their token count
     int64_t suffix_tok_sum;
 };
+
+// Remember e (if it is an error) as the calling thread's last CUDA error.
+cudaError_t note_cuda(cudaError_t e);
 
 }  // namespace fca
 
@@ -87,6 +91,7 @@ struct fca_plan_s {
     int32_t* g_moff = nullptr;
     int32_t* g_nm = nullptr;
     int32_t* g_nch = nullptr;        // split chunks of the group's token range
+    int32_t* g_chunk = nullptr;      // tokens per chunk (last one may be shorter)
     int32_t* g_part = nullptr;       // partial row of (group, head 0, chunk 0, row 0)
     int32_t* members = nullptr;      // [n_member_entries]
     int32_t* suffix_start = nullptr; // [R] blocks
@@ -94,6 +99,8 @@ struct fca_plan_s {
     int32_t* chain_g = nullptr;      // groups of request r, root first
     int32_t* chain_pos = nullptr;    // r's index among the group's members
     int32_t* s_nch = nullptr;        // [R] chunks of r's own pass
+    int32_t* s_chunk = nullptr;      // [R] tokens per chunk (last one may be shorter)
+    int32_t* sched = nullptr;        // [4] work counters of the two passes (self-resetting)
     int32_t* s_part = nullptr;       // [R] partial row of (r, head 0, chunk 0)
     fca::PrefixItem* prefix_items = nullptr;
     fca::SuffixItem* suffix_items = nullptr;

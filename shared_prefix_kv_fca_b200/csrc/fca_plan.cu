@@ -67,6 +67,13 @@ struct PlanScratch {
 
 __device__ __forceinline__ int32_t ceil_div_dev(int32_t a, int32_t b) { return (a + b - 1) / b; }
 
+// Own-pass items are ordered by length (in blocks, capped) so that the
+// longest are taken first.
+constexpr int32_t kBins = 1024;
+__device__ __forceinline__ int32_t length_bin(int32_t tokens) {
+    return min(kBins - 1, (tokens + kBlockSize - 1) / kBlockSize);
+}
+
 // ------------------------------------------------------------ validation
 
 // Thread (r, j): checks seq_lens[r] (j == 0) and table entry j if it is read.
@@ -440,6 +447,10 @@ struct FinalizeArgs {
     int32_t* s_nch;
     int32_t* s_part;
     int32_t* chain_off;  // [R + 1]
+    int32_t* g_chunk;
+    int32_t* s_chunk;
+    int32_t* bin_cursor; // [kBins] first item slot of each length bin, longest first
+    int32_t num_sms;
 };
 
 // One CTA of 1024 threads.  Shared memory: sort keys (next pow2 of R, 8 B)
@@ -495,20 +506,28 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
         A.g_parent[i] = par;
     }
 
-    // split length
+    // Chunk targets.  The grouped pass runs one CTA per SM, so aim at about
+    // three items per SM; the per-request pass runs one item per warp, eight
+    // warps per SM, so aim at about four items per warp.  Each group / request
+    // then splits its tokens evenly into chunks of at most the target.
     const int32_t tile_rows = kPrefixTileRows;
-    int64_t w = 0;
+    int64_t wp = 0, ws = 0;
     for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
         const int64_t tok = (int64_t)(A.g_b[i] - A.g_a[i]) * kBlockSize;
-        w += tok * ((A.g_nm[i] * G + tile_rows - 1) / tile_rows);
+        wp += tok * ((A.g_nm[i] * G + tile_rows - 1) / tile_rows);
     }
     for (int32_t r = threadIdx.x; r < R; r += blockDim.x)
-        w += A.seq_lens[r] - (int64_t)A.suffix_start[r] * kBlockSize;
-    const int64_t work = block_sum64(w, red);
-    int32_t split = A.split_opt;
-    if (split <= 0) {
-        const int64_t target = work / 1184;   // about 8 items per SM over 148 SMs
-        split = (int32_t)std::min<int64_t>(4096, std::max<int64_t>(256, (target + 63) / 64 * 64));
+        ws += A.seq_lens[r] - (int64_t)A.suffix_start[r] * kBlockSize;
+    wp = block_sum64(wp, red) * A.Hkv;
+    ws = block_sum64(ws, red) * A.Hkv;
+    int32_t split_p = A.split_opt, split_s = A.split_opt;
+    if (split_p <= 0) {
+        const int64_t t = wp / (int64_t)(3 * max(1, A.num_sms));
+        split_p = (int32_t)min((int64_t)16384, max((int64_t)512, (t + 63) / 64 * 64));
+    }
+    if (split_s <= 0) {
+        const int64_t t = ws / (int64_t)(32 * max(1, A.num_sms));
+        split_s = (int32_t)min((int64_t)8192, max((int64_t)256, (t + 63) / 64 * 64));
     }
 
     // per-group chunk counts, item offsets, partial bases, member offsets
@@ -516,7 +535,9 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
                                                    A.g_moff, red);
     for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
         const int32_t tok = (A.g_b[i] - A.g_a[i]) * kBlockSize;
-        A.g_nch[i] = (tok + split - 1) / split;
+        const int32_t nch = (tok + split_p - 1) / split_p;
+        A.g_nch[i] = nch;
+        A.g_chunk[i] = ((tok + nch - 1) / nch + kStageTokens - 1) / kStageTokens * kStageTokens;
     }
     __syncthreads();
     const int64_t n_pitems = block_exclusive_scan(
@@ -525,11 +546,32 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
     const int64_t n_ppart = block_exclusive_scan(
         n, [&](int32_t i) { return (int64_t)A.Hkv * A.g_nch[i] * A.g_nm[i] * G; }, A.g_part, red);
 
+    // per-request chunks; own-pass items are binned by length, longest first
+    int32_t* bins = reinterpret_cast<int32_t*>(red + 64 + 1024);
+    for (int32_t b = threadIdx.x; b < kBins; b += blockDim.x) bins[b] = 0;
+    __syncthreads();
     for (int32_t r = threadIdx.x; r < R; r += blockDim.x) {
         const int32_t tok = A.seq_lens[r] - A.suffix_start[r] * kBlockSize;
-        A.s_nch[r] = (tok + split - 1) / split;
+        const int32_t nch = (tok + split_s - 1) / split_s;
+        A.s_nch[r] = nch;
+        const int32_t chunk = nch ? ((tok + nch - 1) / nch + kBlockSize - 1) / kBlockSize * kBlockSize : 0;
+        A.s_chunk[r] = chunk;
+        if (nch) {
+            const int32_t last = tok - (nch - 1) * chunk;
+            atomicAdd(&bins[length_bin(chunk)], A.Hkv * (nch - 1));
+            atomicAdd(&bins[length_bin(last)], A.Hkv);
+        }
     }
     __syncthreads();
+    if (threadIdx.x == 0) {
+        int32_t acc = 0;
+        for (int32_t b = kBins - 1; b >= 0; --b) {
+            A.bin_cursor[b] = acc;
+            acc += bins[b];
+        }
+    }
+    __syncthreads();
+    const int32_t split = split_s;
     const int64_t n_sitems = block_exclusive_scan(R, [&](int32_t r) { return (int64_t)A.Hkv * A.s_nch[r]; },
                                                   A.s.s_item_off, red);
     const int64_t n_spart = block_exclusive_scan(
@@ -555,6 +597,7 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
         hdr->n_member_entries = (int32_t)n_members;
         hdr->max_depth = depth;
         hdr->split_tokens = split;
+        hdr->prefix_split_tokens = split_p;
         hdr->n_prefix_items = (int32_t)n_pitems;
         hdr->n_suffix_items = (int32_t)n_sitems;
         hdr->n_prefix_partials = (int32_t)n_ppart;
@@ -608,15 +651,17 @@ __global__ void __launch_bounds__(256) k_sort_members(const PlanHeader* hdr, con
 // One CTA per group: items (head, q-tile, chunk), heads outermost.
 __global__ void k_fill_prefix_items(const PlanHeader* hdr, const int32_t* g_a, const int32_t* g_b,
                                     const int32_t* g_nm, const int32_t* g_moff, const int32_t* g_nch,
-                                    const int32_t* g_part, const int32_t* item_off, const int32_t* members,
-                                    int32_t G, int32_t Hkv, PrefixItem* items) {
-    const int32_t ng = hdr->n_groups, split = hdr->split_tokens;
+                                    const int32_t* g_chunk, const int32_t* g_part, const int32_t* item_off,
+                                    const int32_t* members, int32_t G, int32_t Hkv, PrefixItem* items) {
+    const int32_t ng = hdr->n_groups;
     for (int32_t g = blockIdx.x; g < ng; g += gridDim.x) {
         const int32_t rows = g_nm[g] * G, tiles = (rows + kPrefixTileRows - 1) / kPrefixTileRows;
-        const int32_t nch = g_nch[g], per_head = tiles * nch;
+        const int32_t nch = g_nch[g], per_head = tiles * nch, split = g_chunk[g];
         const int32_t t0 = g_a[g] * kBlockSize, t1 = g_b[g] * kBlockSize;
+        // heads innermost: the KV heads of one token are neighbours in the cache
+        // (one DRAM row holds all of them), so their items should run together
         for (int32_t i = threadIdx.x; i < Hkv * per_head; i += blockDim.x) {
-            const int32_t h = i / per_head, rem = i % per_head, tile = rem / nch, c = rem % nch;
+            const int32_t h = i % Hkv, rem = i / Hkv, c = rem % nch, tile = rem / nch;
             PrefixItem it;
             it.group = g;
             it.head = h;
@@ -632,22 +677,26 @@ __global__ void k_fill_prefix_items(const PlanHeader* hdr, const int32_t* g_a, c
 }
 
 __global__ void k_fill_suffix_items(int32_t R, const int32_t* seq_lens, const int32_t* suffix_start,
-                                    const int32_t* s_nch, const int32_t* s_part, const int32_t* item_off,
-                                    const PlanHeader* hdr, int32_t G, int32_t Hkv, SuffixItem* items) {
-    const int32_t split = hdr->split_tokens;
+                                    const int32_t* s_nch, const int32_t* s_chunk, const int32_t* s_part,
+                                    int32_t* bin_cursor, int32_t G, int32_t Hkv, SuffixItem* items) {
+    // one thread per request; the Hkv heads of one chunk take consecutive
+    // slots (one DRAM row holds all heads of a token, so they should run together)
     for (int32_t r = blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x) {
-        const int32_t nch = s_nch[r];
+        const int32_t nch = s_nch[r], chunk = s_chunk[r];
         const int32_t t0 = suffix_start[r] * kBlockSize, L = seq_lens[r];
-        for (int32_t i = 0; i < Hkv * nch; ++i) {
-            const int32_t h = i / nch, c = i % nch;
-            SuffixItem it;
-            it.request = r;
-            it.head = h;
-            it.tok0 = t0 + c * split;
-            it.tok1 = min(L, it.tok0 + split);
-            it.part_row0 = s_part[r] + (h * nch + c) * G;
-            it.pad0 = it.pad1 = it.pad2 = 0;
-            items[item_off[r] + i] = it;
+        for (int32_t c = 0; c < nch; ++c) {
+            const int32_t tok0 = t0 + c * chunk, tok1 = min(L, tok0 + chunk);
+            const int32_t pos = atomicAdd(&bin_cursor[length_bin(tok1 - tok0)], Hkv);
+            for (int32_t h = 0; h < Hkv; ++h) {
+                SuffixItem it;
+                it.request = r;
+                it.head = h;
+                it.tok0 = tok0;
+                it.tok1 = tok1;
+                it.part_row0 = s_part[r] + (h * nch + c) * G;
+                it.pad0 = it.pad1 = it.pad2 = 0;
+                items[pos + h] = it;
+            }
         }
     }
 }
@@ -680,7 +729,7 @@ template <typename T>
 T* plan_alloc(fca_plan_s* P, size_t count, bool& ok) {
     void* p = nullptr;
     const size_t bytes = std::max<size_t>(count, 1) * sizeof(T);
-    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+    if (note_cuda(cudaMalloc(&p, bytes)) != cudaSuccess) {
         ok = false;
         (void)cudaGetLastError();
         return nullptr;
@@ -705,7 +754,7 @@ int32_t next_pow2(int32_t n) {
 
 #define FCA_CK(x)                                \
     do {                                         \
-        if ((x) != cudaSuccess) {                \
+        if (note_cuda(x) != cudaSuccess) {       \
             (void)cudaGetLastError();            \
             return FCA_ERR_CUDA;                 \
         }                                        \
@@ -748,6 +797,10 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     P->g_part = plan_alloc<int32_t>(P, R + 1, ok);
     P->s_nch = plan_alloc<int32_t>(P, R, ok);
     P->s_part = plan_alloc<int32_t>(P, R + 1, ok);
+    P->g_chunk = plan_alloc<int32_t>(P, R, ok);
+    P->s_chunk = plan_alloc<int32_t>(P, R, ok);
+    P->sched = plan_alloc<int32_t>(P, 4, ok);
+    int32_t* bin_cursor = tmp.alloc<int32_t>(kBins);
     P->chain_off = plan_alloc<int32_t>(P, R + 1, ok);
     P->dev_status = plan_alloc<int32_t>(P, 1, ok);
     if (!ok) return FCA_ERR_OOM;
@@ -766,6 +819,7 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     FCA_CK(cudaMemsetAsync(s.hdr, 0, sizeof(PlanHeader), stream));
     FCA_CK(cudaMemsetAsync(P->suffix_start, 0, sizeof(int32_t) * R, stream));
     FCA_CK(cudaMemsetAsync(P->dev_status, 0, sizeof(int32_t), stream));
+    FCA_CK(cudaMemsetAsync(P->sched, 0, 4 * sizeof(int32_t), stream));
 
     const int64_t cells = (int64_t)R * max_blocks;
     k_validate<<<grid_for(cells, 256), 256, 0, stream>>>(P->bt, max_blocks, P->seq_lens, R, num_blocks, s.nfull,
@@ -818,7 +872,16 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     fa.s_nch = P->s_nch;
     fa.s_part = P->s_part;
     fa.chain_off = P->chain_off;
-    const size_t fin_smem = (size_t)next_pow2(R) * 8 + (64 + 1024) * 8;
+    fa.g_chunk = P->g_chunk;
+    fa.s_chunk = P->s_chunk;
+    fa.bin_cursor = bin_cursor;
+    {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        fa.num_sms = 148;
+        cudaDeviceGetAttribute(&fa.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const size_t fin_smem = (size_t)next_pow2(R) * 8 + (64 + 1024) * 8 + kBins * 4;
     FCA_CK(cudaFuncSetAttribute(k_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem));
     k_finalize<<<1, 1024, fin_smem, stream>>>(fa);
     FCA_CK(cudaGetLastError());
@@ -857,14 +920,13 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
         k_sort_members<<<std::min(H.n_groups, 148 * 4), 256, mem_smem, stream>>>(
             s.hdr, P->g_moff, P->g_nm, P->members, P->chain_off, P->chain_g, P->chain_pos);
         k_fill_prefix_items<<<std::min(H.n_groups, 148 * 4), 256, 0, stream>>>(
-            s.hdr, P->g_a, P->g_b, P->g_nm, P->g_moff, P->g_nch, P->g_part, s.g_item_off, P->members, G, Hkv,
-            P->prefix_items);
+            s.hdr, P->g_a, P->g_b, P->g_nm, P->g_moff, P->g_nch, P->g_chunk, P->g_part, s.g_item_off, P->members,
+            G, Hkv, P->prefix_items);
         FCA_CK(cudaGetLastError());
     }
     if (H.n_suffix_items > 0) {
-        k_fill_suffix_items<<<grid_for(R, 128), 128, 0, stream>>>(R, P->seq_lens, P->suffix_start, P->s_nch,
-                                                                  P->s_part, s.s_item_off, s.hdr, G, Hkv,
-                                                                  P->suffix_items);
+        k_fill_suffix_items<<<grid_for(R, 128), 128, 0, stream>>>(
+            R, P->seq_lens, P->suffix_start, P->s_nch, P->s_chunk, P->s_part, bin_cursor, G, Hkv, P->suffix_items);
         FCA_CK(cudaGetLastError());
     }
     return FCA_OK;   // temporaries go back to the pool in stream order

@@ -8,24 +8,36 @@
 // into one 128-row Q tile, which turns the pass into a dense contraction
 // against the shared K and V.
 //
-// One CTA per work item = (group, KV head, 128-row Q tile, token chunk); 192
-// threads in three roles:
-//   warp 0      TMA producer: streams 64-token stages of K and V (four paged
-//               16-token blocks, two 64-column halves each, 128-byte swizzle)
-//               into a ring of kPreStages slots; blocks past the chunk are
-//               loaded from out-of-range rows, i.e. as zeros;
+// Work item = (group, KV head, 128-row Q tile, token chunk).  The kernel is
+// persistent: one CTA per SM walks its items (blockIdx.x, +gridDim.x, ...),
+// tensor memory is allocated once, and the K/V stream runs on across items.
+// 320 threads in three roles:
+//   warp 0      TMA producer: 64-token stages of K and V (four paged 16-token
+//               blocks, 64-column halves, 128-byte swizzle) into a ring of
+//               kPreStages slots; blocks past a chunk are loaded from rows
+//               beyond the cache, which TMA fills with zeros;
 //   warp 1      allocates tensor memory and, from one thread, issues
-//               S = Q K^T (M=128, N=64, K=head_dim) into one of two S buffers
-//               and O_s = P V (M=128, N=head_dim, K=64) into one of two O
-//               buffers, signalling completions with tcgen05.commit;
-//   warps 2-5   softmax: thread = query row (TMEM lane); read the S row,
-//               online max / sum in fp32 (log2 domain), write P as bf16 into
-//               shared memory in the MMA's K-major swizzled layout, then fold
-//               the previous stage's O_s into a register accumulator with the
-//               running rescale factor.
-// The S buffer of stage j+1 is computed while stage j's softmax runs.
+//               S = Q K^T (M=128, N=64) and O_w += P V (M=128, N=head_dim),
+//               signalling completions with tcgen05.commit.  Q and P are the
+//               A operands and live in tensor memory next to S and O, so all
+//               of shared memory holds the K/V ring (the stages a slow HBM
+//               stream needs in flight); a K slot is released as soon as its
+//               Q K^T has run, a V slot after its P V;
+//   warps 2-9   two softmax warpgroups, one thread per query row each.  Stage
+//               s of an item belongs to warpgroup s % 2, which has its own S
+//               buffer, P buffer, O accumulator and online-softmax state, so
+//               the two groups work on consecutive stages at the same time
+//               and never wait for each other inside an item.  fp32 max in
+//               the log2 domain; P stored to tensor memory as packed bf16.  A group's O accumulator is rescaled in
+//               tensor memory only when a row's maximum grows by more than
+//               2^kRescaleLog2 over the one its exponentials use, which after
+//               the first stages is rare (numerator and denominator use the
+//               same reference, so the result is exact).  At the end of an
+//               item the two partial states are merged by their weights.
 // Output: one partial row (normalised o, natural-log lse) per stacked query
 // row, merged later with the row's other partials.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 
 #include "fca_device.cuh"
@@ -35,16 +47,21 @@ namespace fca {
 
 namespace {
 
-constexpr int kPreStages = 4;
-constexpr int kPreThreads = 192;
+constexpr int kPreStages = 6;
+constexpr int kSoftWarps = 8;
+constexpr int kPreThreads = 64 + kSoftWarps * 32;
+constexpr float kRescaleLog2 = 8.f;
 
 struct PrefixArgs {
     const PrefixItem* items;
+    int32_t n_items;
     const int32_t* bt;
     const int32_t* members;
     const int32_t* g_moff;
-    int32_t max_blocks, num_blocks, Hq, G;
+    int32_t max_blocks, num_blocks, Hq, G, Hkv;
     const __nv_bfloat16* q;
+    const uint8_t* k_cache;   // raw cache bases, for whole-block L2 prefetch
+    const uint8_t* v_cache;
     float scale_log2;
     float* part_o;
     float* part_lse;
@@ -54,23 +71,27 @@ struct PrefixArgs {
 template <int D>
 struct PreLayout {
     static constexpr int kHalves = D / 64;
-    static constexpr int kQ = kHalves * 128 * 128;        // Q tile, bytes
     static constexpr int kKV = kHalves * 64 * 128;        // one 64-token K (or V) stage
-    static constexpr int kP = 128 * 128;                  // one P buffer (128 rows x 64 bf16)
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kQ;
+    static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kPreStages * kKV;
-    static constexpr int kOffP = kOffV + kPreStages * kKV;
-    static constexpr int kOffBar = kOffP + 2 * kP;
-    // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], s_free[2],
-    //           p_full[2], o_full[2], o_free[2], mma_done
-    static constexpr int kNumBars = 1 + 3 * kPreStages + 10 + 1;
+    static constexpr int kOffX = kOffV + kPreStages * kKV; // per-row (m, l) of each group [2 items][2][2][128] f32
+    static constexpr int kOffBar = kOffX + 2 * 2 * 2 * 128 * 4;
+    // q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], s_free[2],
+    // p_full[2], p_free[2], o_full[2], o_free, mma_done, l_bar
+    static constexpr int kNumBars = 1 + 4 * kPreStages + 10 + 3;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kTotal = kOffMisc + 64 + 1024;   // + alignment slack
-    static constexpr uint32_t kTmemCols = D == 128 ? 512 : 256;
-    static constexpr uint32_t kColS = 0;                  // two 64-column S buffers
-    static constexpr uint32_t kColO = 128;                // two D-column O buffers
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColS = 0;                  // S of group w: 64 fp32 columns at 64 w
+    static constexpr uint32_t kColO = 128;                // O of group w: D fp32 columns at 128 + D w
+    static constexpr uint32_t kColP = 128 + 2 * D;        // P of group w: 32 columns (64 bf16) at + 32 w
+    static constexpr uint32_t kColQ = kColP + 64;         // Q: D / 2 columns (D bf16)
+    static_assert(kColQ + D / 2 <= kTmemCols, "tensor memory budget");
 };
+
+__device__ __forceinline__ int32_t stages_of(const PrefixItem& it) {
+    return (it.tok1 - it.tok0 + kStageTokens - 1) / kStageTokens;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kPreThreads, 1)
@@ -82,36 +103,41 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;
     uint64_t* v_full = k_full + kPreStages;
-    uint64_t* kv_empty = v_full + kPreStages;
-    uint64_t* s_full = kv_empty + kPreStages;
+    uint64_t* k_empty = v_full + kPreStages;
+    uint64_t* v_empty = k_empty + kPreStages;
+    uint64_t* s_full = v_empty + kPreStages;
     uint64_t* s_free = s_full + 2;
     uint64_t* p_full = s_free + 2;
-    uint64_t* o_full = p_full + 2;
+    uint64_t* p_free = p_full + 2;
+    uint64_t* o_full = p_free + 2;
     uint64_t* o_free = o_full + 2;
-    uint64_t* mma_done = o_free + 2;
+    uint64_t* mma_done = o_free + 1;
+    uint64_t* l_bar = mma_done + 1;      // end-of-item exchange of (m, l) between the groups
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 16);
+    float* xml = reinterpret_cast<float*>(smem + L::kOffX);
 
-    const PrefixItem it = a.items[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int32_t n_tok = it.tok1 - it.tok0;
-    const int32_t n_stages = (n_tok + kStageTokens - 1) / kStageTokens;
+    const int32_t first_item = blockIdx.x, item_step = gridDim.x;
 
     if (threadIdx.x == 0) {
         dev::mbar_init(q_full, 128);
-        for (int s = 0; s < kPreStages; ++s) {
-            dev::mbar_init(&k_full[s], 1);
-            dev::mbar_init(&v_full[s], 1);
-            dev::mbar_init(&kv_empty[s], 1);
+        for (int st = 0; st < kPreStages; ++st) {
+            dev::mbar_init(&k_full[st], 1);
+            dev::mbar_init(&v_full[st], 1);
+            dev::mbar_init(&k_empty[st], 1);
+            dev::mbar_init(&v_empty[st], 1);
         }
         for (int b = 0; b < 2; ++b) {
             dev::mbar_init(&s_full[b], 1);
             dev::mbar_init(&s_free[b], 128);
             dev::mbar_init(&p_full[b], 128);
+            dev::mbar_init(&p_free[b], 1);
             dev::mbar_init(&o_full[b], 1);
-            dev::mbar_init(&o_free[b], 128);
         }
+        dev::mbar_init(o_free, kSoftWarps * 32);
         dev::mbar_init(mma_done, 1);
+        dev::mbar_init(l_bar, kSoftWarps * 32);
         *abort_flag = 0;
         dev::fence_mbarrier_init();
     }
@@ -126,40 +152,80 @@ __global__ void __launch_bounds__(kPreThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
+        // The whole warp fetches block ids, 32 at a time (eight stages' worth)
+        // and one batch ahead, so no table lookup sits on the issue path;
+        // lane 0 waits for free slots and issues the copies.
+        constexpr int kBlkPerStage = kStageTokens / kBlockSize;
+        constexpr int kStagesPerBatch = 32 / kBlkPerStage;
         if (lane == 0) {
             dev::tma_prefetch_desc(&tmK);
             dev::tma_prefetch_desc(&tmV);
+        }
+        uint32_t g = 0;
+        bool ok = true;
+        int32_t pending_k = -1;     // stage whose K copies are in flight but whose V is not issued
+        for (int32_t item = first_item; ok && item < a.n_items; item += item_step) {
+            const PrefixItem it = a.items[item];
             const int32_t* row = a.bt + (int64_t)it.bt_row * a.max_blocks;
             const int32_t blk0 = it.tok0 / kBlockSize, blk_end = it.tok1 / kBlockSize;
-            int32_t issued = 0;
-            for (int32_t j = 0; j < n_stages; ++j) {
-                const int s = j % kPreStages;
-                if (j >= kPreStages &&
-                    !dev::mbar_wait(&kv_empty[s], ((j / kPreStages) - 1) & 1, abort_flag, a.err))
-                    break;
-                uint8_t* kdst = smem + L::kOffK + s * L::kKV;
-                uint8_t* vdst = smem + L::kOffV + s * L::kKV;
-                dev::mbar_arrive_expect_tx(&k_full[s], L::kKV);
-                dev::mbar_arrive_expect_tx(&v_full[s], L::kKV);
+            const int32_t ns = stages_of(it);
+            auto fetch = [&](int32_t batch) -> int32_t {
+                const int32_t blk = blk0 + batch * 32 + lane;
+                // past the chunk: rows beyond the cache, which TMA fills with zeros
+                return blk < blk_end ? __ldg(row + blk) * kBlockSize : a.num_blocks * kBlockSize;
+            };
+            int32_t nxt = fetch(0), cur = 0;
+            for (int32_t j = 0; j < ns; ++j, ++g) {
+                if (j % kStagesPerBatch == 0) {
+                    cur = nxt;
+                    nxt = fetch(j / kStagesPerBatch + 1);
+                }
+                int32_t trow[kBlkPerStage];
 #pragma unroll
-                for (int bi = 0; bi < kStageTokens / kBlockSize; ++bi) {
-                    const int32_t blk = blk0 + j * (kStageTokens / kBlockSize) + bi;
-                    // past the chunk: rows beyond the cache, which TMA fills with zeros
-                    const int32_t trow = blk < blk_end ? row[blk] * kBlockSize : a.num_blocks * kBlockSize;
+                for (int bi = 0; bi < kBlkPerStage; ++bi)
+                    trow[bi] = __shfl_sync(0xffffffffu, cur, (j % kStagesPerBatch) * kBlkPerStage + bi);
+                if (lane == 0) {
+                    const int s = g % kPreStages;
+                    const uint32_t ph = ((g / kPreStages) - 1) & 1;
+                    uint8_t* kdst = smem + L::kOffK + s * L::kKV;
+                    uint8_t* vdst = smem + L::kOffV + s * L::kKV;
+                    if (g >= kPreStages && !dev::mbar_wait(&k_empty[s], ph, abort_flag, a.err)) {
+                        ok = false;
+                    } else {
+                        dev::mbar_arrive_expect_tx(&k_full[s], L::kKV);
 #pragma unroll
-                    for (int hf = 0; hf < L::kHalves; ++hf) {
-                        dev::tma_load_3d(kdst + hf * (64 * 128) + bi * 2048, &tmK, &k_full[s], hf * 64, it.head,
-                                         trow);
-                        dev::tma_load_3d(vdst + hf * (64 * 128) + bi * 2048, &tmV, &v_full[s], hf * 64, it.head,
-                                         trow);
+                        for (int bi = 0; bi < kBlkPerStage; ++bi)
+#pragma unroll
+                            for (int hf = 0; hf < L::kHalves; ++hf)
+                                dev::tma_load_3d(kdst + hf * (64 * 128) + bi * 2048, &tmK, &k_full[s], hf * 64,
+                                                 it.head, trow[bi]);
+                        pending_k = (int32_t)g;
+                        if (g >= kPreStages && !dev::mbar_wait(&v_empty[s], ph, abort_flag, a.err)) {
+                            ok = false;
+                        } else {
+                            dev::mbar_arrive_expect_tx(&v_full[s], L::kKV);
+#pragma unroll
+                            for (int bi = 0; bi < kBlkPerStage; ++bi)
+#pragma unroll
+                                for (int hf = 0; hf < L::kHalves; ++hf)
+                                    dev::tma_load_3d(vdst + hf * (64 * 128) + bi * 2048, &tmV, &v_full[s], hf * 64,
+                                                     it.head, trow[bi]);
+                            pending_k = -1;
+                        }
                     }
                 }
-                ++issued;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
             }
-            for (int32_t j = issued - 1; j >= 0 && j >= issued - kPreStages; --j) {
-                volatile int never = 0;
-                dev::mbar_wait(&k_full[j % kPreStages], (j / kPreStages) & 1, &never, a.err);
-                dev::mbar_wait(&v_full[j % kPreStages], (j / kPreStages) & 1, &never, a.err);
+        }
+        if (lane == 0) {
+            // never leave with copies in flight
+            volatile int never = 0;
+            if (pending_k >= 0)
+                dev::mbar_wait(&k_full[pending_k % kPreStages], (pending_k / kPreStages) & 1, &never, a.err);
+            for (uint32_t j = g; j > 0 && j + kPreStages > g; --j) {
+                dev::mbar_wait(&k_full[(j - 1) % kPreStages], ((j - 1) / kPreStages) & 1, &never, a.err);
+                dev::mbar_wait(&v_full[(j - 1) % kPreStages], ((j - 1) / kPreStages) & 1, &never, a.err);
             }
         }
         __syncwarp();
@@ -168,41 +234,62 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = dev::idesc_bf16_f32(128, 64, false, false);
             constexpr uint32_t idesc_pv = dev::idesc_bf16_f32(128, D, false, true);
-            const uint32_t q_base = dev::smem_u32(smem + L::kOffQ);
-            bool ok = dev::mbar_wait(q_full, 0, abort_flag, a.err);
-            auto issue_qk = [&](int32_t j) -> bool {
-                const int s = j % kPreStages, sb = j & 1;
-                if (!dev::mbar_wait(&k_full[s], (j / kPreStages) & 1, abort_flag, a.err)) return false;
-                if (j >= 2 && !dev::mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1, abort_flag, a.err)) return false;
+            auto issue_qk = [&](uint32_t gg) -> bool {
+                const int s = gg % kPreStages, sb = gg & 1;
+                if (!dev::mbar_wait(&k_full[s], (gg / kPreStages) & 1, abort_flag, a.err)) return false;
+                if (gg >= 2 && !dev::mbar_wait(&s_free[sb], ((gg >> 1) - 1) & 1, abort_flag, a.err)) return false;
                 dev::tc_fence_after();
                 const uint32_t k_base = dev::smem_u32(smem + L::kOffK + s * L::kKV);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint64_t ad = dev::smem_desc_sw128(q_base + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024);
-                    const uint64_t bd = dev::smem_desc_sw128(k_base + (k >> 2) * (64 * 128) + (k & 3) * 32, 16, 1024);
-                    dev::tc_mma_ss(tmem + L::kColS + sb * 64, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+                    const uint64_t bd =
+                        dev::smem_desc_sw128(k_base + (k >> 2) * (64 * 128) + (k & 3) * 32, 16, 1024);
+                    dev::tc_mma_ts(tmem + L::kColS + sb * 64, tmem + L::kColQ + k * 8, bd, idesc_qk, k > 0 ? 1u : 0u);
                 }
                 dev::tc_commit(&s_full[sb]);
+                dev::tc_commit(&k_empty[s]);
                 return true;
             };
-            if (ok && n_stages > 0) ok = issue_qk(0);
-            for (int32_t j = 0; ok && j < n_stages; ++j) {
-                if (j + 1 < n_stages && !issue_qk(j + 1)) { ok = false; break; }
-                const int s = j % kPreStages, pb = j & 1;
-                if (!dev::mbar_wait(&p_full[pb], (j >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
-                if (j >= 2 && !dev::mbar_wait(&o_free[pb], ((j >> 1) - 1) & 1, abort_flag, a.err)) { ok = false; break; }
-                if (!dev::mbar_wait(&v_full[s], (j / kPreStages) & 1, abort_flag, a.err)) { ok = false; break; }
+            // first: the first P V of group (gg & 1) in this item, which starts
+            // its O accumulator afresh once the previous item's epilogue read it
+            auto issue_pv = [&](uint32_t gg, bool first, int32_t local_item) -> bool {
+                const int s = gg % kPreStages, pb = gg & 1;
+                if (!dev::mbar_wait(&p_full[pb], (gg >> 1) & 1, abort_flag, a.err)) return false;
+                if (first && local_item > 0 && !dev::mbar_wait(o_free, (local_item - 1) & 1, abort_flag, a.err))
+                    return false;
+                if (!dev::mbar_wait(&v_full[s], (gg / kPreStages) & 1, abort_flag, a.err)) return false;
                 dev::tc_fence_after();
-                const uint32_t p_base = dev::smem_u32(smem + L::kOffP + pb * L::kP);
                 const uint32_t v_base = dev::smem_u32(smem + L::kOffV + s * L::kKV);
 #pragma unroll
                 for (int k = 0; k < kStageTokens / 16; ++k) {
-                    const uint64_t ad = dev::smem_desc_sw128(p_base + k * 32, 16, 1024);
                     const uint64_t bd = dev::smem_desc_sw128(v_base + k * 2048, 64 * 128, 1024);
-                    dev::tc_mma_ss(tmem + L::kColO + pb * D, ad, bd, idesc_pv, k > 0 ? 1u : 0u);
+                    dev::tc_mma_ts(tmem + L::kColO + pb * D, tmem + L::kColP + pb * 32 + k * 8, bd, idesc_pv,
+                                   (first && k == 0) ? 0u : 1u);
                 }
                 dev::tc_commit(&o_full[pb]);
-                dev::tc_commit(&kv_empty[s]);
+                dev::tc_commit(&p_free[pb]);
+                dev::tc_commit(&v_empty[s]);
+                return true;
+            };
+            bool ok = true;
+            uint32_t g = 0;
+            int32_t local = 0;
+            if (first_item < a.n_items) ok = dev::mbar_wait(q_full, 0, abort_flag, a.err) && issue_qk(0);
+            for (int32_t item = first_item; ok && item < a.n_items; item += item_step, ++local) {
+                const int32_t ns = stages_of(a.items[item]);
+                const bool has_next = item + item_step < a.n_items;
+                for (int32_t j = 0; ok && j < ns; ++j) {
+                    const uint32_t gg = g + j;
+                    if (j + 1 < ns) {
+                        ok = issue_qk(gg + 1) && issue_pv(gg, j < 2, local);
+                    } else {
+                        // last stage: finish this item's O first, then start the next item
+                        ok = issue_pv(gg, j < 2, local);
+                        if (ok && has_next)
+                            ok = dev::mbar_wait(q_full, (local + 1) & 1, abort_flag, a.err) && issue_qk(gg + 1);
+                    }
+                }
+                g += ns;
             }
             // every MMA of this thread has retired before tensor memory is freed
             dev::tc_commit(mma_done);
@@ -211,114 +298,180 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ softmax warps
-        const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
-        const int r = quarter * 32 + lane;            // tile row
+        // ------------------------------------------------ softmax warpgroups
+        const int quarter = warp & 3;                  // TMEM lane quarter of this warp
+        const int wg = (warp - 2) >> 2;                // stages of parity wg are this group's
+        const int r = quarter * 32 + lane;             // tile row
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const bool row_valid = r < it.nrows;
+        const uint32_t s_col = L::kColS + wg * 64, o_col = L::kColO + wg * D;
+        constexpr int kOHalf = D / 2;
 
-        // Q tile row r: stacked row it.row0 + r = member (i / G), query head (head * G + i % G)
-        {
-            uint8_t* qdst = smem + L::kOffQ;
-            const __nv_bfloat16* src = nullptr;
-            if (row_valid) {
+        // Q tile row r (whole row): stacked row row0 + r = member (i / G),
+        // query head head * G + i % G; rows past the tile are zero.
+        auto load_q = [&](const PrefixItem& it) {
+            const bool valid = r < it.nrows;
+            const uint4* src = nullptr;
+            if (valid) {
                 const int32_t i = it.row0 + r;
                 const int32_t member = a.members[a.g_moff[it.group] + i / a.G];
-                src = a.q + ((int64_t)member * a.Hq + it.head * a.G + i % a.G) * D;
+                src = reinterpret_cast<const uint4*>(a.q + ((int64_t)member * a.Hq + it.head * a.G + i % a.G) * D);
             }
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (row_valid) v = *reinterpret_cast<const uint4*>(src + c * 8);
-                const int hf = c >> 3, cc = c & 7;
-                *reinterpret_cast<uint4*>(qdst + hf * (128 * 128) + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
-            }
-            dev::fence_proxy_async_smem();
-            dev::mbar_arrive(q_full);
-        }
-
-        float m_run = -INFINITY, l_run = 0.f, alpha_last = 0.f;
-        float oacc[D];
-#pragma unroll
-        for (int d = 0; d < D; ++d) oacc[d] = 0.f;
-        bool ok = true;
-
-        auto fold = [&](int32_t jj, float al) -> bool {
-            const int ob = jj & 1;
-            const bool got = dev::mbar_wait(&o_full[ob], (jj >> 1) & 1, abort_flag, a.err);
-            if (!__all_sync(0xffffffffu, got)) return false;     // tcgen05.ld needs the whole warp
-            dev::tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32];
-                dev::tmem_ld32(tmem + lane_base + L::kColO + ob * D + c * 32, v);
-                dev::tc_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) oacc[c * 32 + i] = fmaf(oacc[c * 32 + i], al, __uint_as_float(v[i]));
-            }
-            dev::tc_fence_before();
-            dev::mbar_arrive(&o_free[ob]);
-            return true;
-        };
-
-        for (int32_t j = 0; j < n_stages; ++j) {
-            const int sb = j & 1;
-            const bool got = dev::mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag, a.err);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-            dev::tc_fence_after();
-            uint32_t s_lo[32], s_hi[32];
-            dev::tmem_ld32(tmem + lane_base + L::kColS + sb * 64, s_lo);
-            dev::tmem_ld32(tmem + lane_base + L::kColS + sb * 64 + 32, s_hi);
-            dev::tc_wait_ld();
-            dev::tc_fence_before();
-            dev::mbar_arrive(&s_free[sb]);
-
-            const int32_t n_valid = min(kStageTokens, n_tok - j * kStageTokens);
-            float sv[64];
-            float mx = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const float raw = __uint_as_float(i < 32 ? s_lo[i & 31] : s_hi[i & 31]);
-                const float x = i < n_valid ? raw * a.scale_log2 : -INFINITY;
-                sv[i] = x;
-                mx = fmaxf(mx, x);
-            }
-            const float m_new = fmaxf(m_run, mx);
-            const float alpha = exp2f(m_run - m_new);
-            float psum = 0.f;
-            uint8_t* prow = smem + L::kOffP + sb * L::kP + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float p[8];
+            for (int c = 0; c < D / 64; ++c) {
+                uint32_t w[32];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    p[e] = exp2f(sv[c * 8 + e] - m_new);
-                    psum += p[e];
+                    const uint4 v = valid ? src[c * 8 + e] : make_uint4(0, 0, 0, 0);
+                    w[e * 4 + 0] = v.x;
+                    w[e * 4 + 1] = v.y;
+                    w[e * 4 + 2] = v.z;
+                    w[e * 4 + 3] = v.w;
                 }
-                uint4 packed;
-                packed.x = dev::pack_bf16x2(p[0], p[1]);
-                packed.y = dev::pack_bf16x2(p[2], p[3]);
-                packed.z = dev::pack_bf16x2(p[4], p[5]);
-                packed.w = dev::pack_bf16x2(p[6], p[7]);
-                *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = packed;
+                dev::tmem_st32(tmem + lane_base + L::kColQ + c * 32, w);
             }
-            l_run = l_run * alpha + psum;
-            m_run = m_new;
-            dev::fence_proxy_async_smem();
-            dev::mbar_arrive(&p_full[sb]);
-            if (j > 0 && !fold(j - 1, alpha_last)) { ok = false; break; }
-            alpha_last = alpha;
-        }
-        if (ok && n_stages > 0) ok = fold(n_stages - 1, alpha_last);
+            dev::tc_wait_st();
+            dev::tc_fence_before();
+            dev::mbar_arrive(q_full);
+        };
 
-        if (ok && row_valid) {
-            const float inv = 1.f / l_run;
-            float* dst = a.part_o + ((int64_t)it.part_row0 + r) * D;
+        bool ok = true;
+        uint32_t g = 0;
+        int32_t local = 0;
+        if (wg == 0 && first_item < a.n_items) load_q(a.items[first_item]);
+        for (int32_t item = first_item; ok && item < a.n_items; item += item_step, ++local) {
+            const PrefixItem it = a.items[item];
+            const int32_t ns = stages_of(it), n_tok = it.tok1 - it.tok0;
+            const bool has_next = item + item_step < a.n_items;
+            float m_ref = -INFINITY, l_run = 0.f;
+            int32_t my_last = -1;                      // my last stage of this item (global index)
+            for (int32_t j = ((g & 1) == (uint32_t)wg) ? 0 : 1; j < ns; j += 2) {
+                const uint32_t gg = g + j;
+                my_last = (int32_t)gg;
+                bool got = dev::mbar_wait(&s_full[wg], (gg >> 1) & 1, abort_flag, a.err);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                dev::tc_fence_after();
+                const int32_t n_valid = min(kStageTokens, n_tok - j * kStageTokens);
+                float x[64];
 #pragma unroll
-            for (int d = 0; d < D; d += 4)
-                *reinterpret_cast<float4*>(dst + d) =
-                    make_float4(oacc[d] * inv, oacc[d + 1] * inv, oacc[d + 2] * inv, oacc[d + 3] * inv);
-            a.part_lse[it.part_row0 + r] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t t[32];
+                    dev::tmem_ld32(tmem + lane_base + s_col + h2 * 32, t);
+                    dev::tc_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        x[h2 * 32 + i] = h2 * 32 + i < n_valid ? __uint_as_float(t[i]) * a.scale_log2 : -INFINITY;
+                }
+                dev::tc_fence_before();
+                dev::mbar_arrive(&s_free[wg]);
+                float mx8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx8[i] = x[i];
+#pragma unroll
+                for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], x[i]);
+                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+
+                float alpha = 1.f;
+                bool rescale = false;
+                if (m_ref == -INFINITY) {
+                    m_ref = mx;                       // this group's first stage of the item
+                } else if (mx > m_ref + kRescaleLog2) {
+                    alpha = dev::ex2(m_ref - mx);
+                    m_ref = mx;
+                    rescale = true;
+                }
+                l_run *= alpha;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // the accumulator may be touched only after this group's previous P V retired
+                    got = dev::mbar_wait(&o_full[wg], ((gg >> 1) - 1) & 1, abort_flag, a.err);
+                    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                    dev::tc_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < D / 16; ++c) {
+                        uint32_t ov[16];
+                        const uint32_t ta = tmem + lane_base + o_col + c * 16;
+                        dev::tmem_ld16(ta, ov);
+                        dev::tc_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                        dev::tmem_st16(ta, ov);
+                    }
+                    dev::tc_wait_st();
+                    dev::tc_fence_before();
+                }
+                if (gg >= 2) {
+                    got = dev::mbar_wait(&p_free[wg], ((gg >> 1) - 1) & 1, abort_flag, a.err);
+                    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                }
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t pw[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float p0 = dev::ex2(x[2 * i] - m_ref), p1 = dev::ex2(x[2 * i + 1] - m_ref);
+                    ls[(2 * i) & 3] += p0;
+                    ls[(2 * i + 1) & 3] += p1;
+                    pw[i] = dev::pack_bf16x2(p0, p1);
+                }
+                l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                dev::tmem_st32(tmem + lane_base + L::kColP + wg * 32, pw);
+                dev::tc_wait_st();
+                dev::tc_fence_before();
+                dev::mbar_arrive(&p_full[wg]);
+                // the group that read the item's last S knows every Q K^T of the
+                // item has completed: it refills the Q tile for the next item
+                if (j + 1 == ns && has_next) load_q(a.items[item + item_step]);
+            }
+            if (!ok) break;
+            g += ns;
+
+            // epilogue: wait for this group's last P V, swap (m, l) with the other
+            // group, and write half of the columns of the merged, normalised rows
+            if (my_last >= 0) {
+                bool got = dev::mbar_wait(&o_full[wg], ((uint32_t)my_last >> 1) & 1, abort_flag, a.err);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            }
+            // (double-buffered by item: the other group may already be writing the next item's)
+            float* xb = xml + (local & 1) * 512;
+            xb[(wg * 2 + 0) * 128 + r] = m_ref;
+            xb[(wg * 2 + 1) * 128 + r] = l_run;
+            dev::mbar_arrive(l_bar);
+            {
+                bool got = dev::mbar_wait(l_bar, local & 1, abort_flag, a.err);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            }
+            dev::tc_fence_after();
+            const float m0 = xb[0 * 128 + r], l0 = xb[1 * 128 + r];
+            const float m1 = xb[2 * 128 + r], l1 = xb[3 * 128 + r];
+            const float m = fmaxf(m0, m1);
+            const float w0 = l0 > 0.f ? dev::ex2(m0 - m) : 0.f, w1 = l1 > 0.f ? dev::ex2(m1 - m) : 0.f;
+            const float l_tot = l0 * w0 + l1 * w1;
+            const float inv = 1.f / l_tot, c0 = w0 * inv, c1 = w1 * inv;
+            const bool row_valid = r < it.nrows;
+            float* dst = a.part_o + ((int64_t)it.part_row0 + r) * D + wg * kOHalf;
+#pragma unroll
+            for (int c = 0; c < kOHalf / 16; ++c) {
+                uint32_t o0[16], o1[16];
+                dev::tmem_ld16(tmem + lane_base + L::kColO + wg * kOHalf + c * 16, o0);
+                dev::tmem_ld16(tmem + lane_base + L::kColO + D + wg * kOHalf + c * 16, o1);
+                dev::tc_wait_ld();
+                if (row_valid) {
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4) {
+                        float v[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float a0 = l0 > 0.f ? __uint_as_float(o0[i + e]) * c0 : 0.f;
+                            const float a1 = l1 > 0.f ? __uint_as_float(o1[i + e]) * c1 : 0.f;
+                            v[e] = a0 + a1;
+                        }
+                        *reinterpret_cast<float4*>(dst + c * 16 + i) = make_float4(v[0], v[1], v[2], v[3]);
+                    }
+                }
+            }
+            dev::tc_fence_before();
+            dev::mbar_arrive(o_free);
+            if (wg == 0 && row_valid)
+                a.part_lse[it.part_row0 + r] = (m + __log2f(l_tot)) * 0.69314718055994531f;
         }
     }
 
@@ -331,23 +484,27 @@ __global__ void __launch_bounds__(kPreThreads, 1)
 }
 
 template <int D>
-cudaError_t launch_prefix_t(const PrefixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int n_items,
-                            cudaStream_t stream) {
+cudaError_t launch_prefix_t(const PrefixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
     using L = PreLayout<D>;
     cudaError_t e = cudaFuncSetAttribute(k_prefix<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
     if (e != cudaSuccess) return e;
-    k_prefix<D><<<n_items, kPreThreads, L::kTotal, stream>>>(a, tk, tv);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = std::max(1, std::min(sms, a.n_items));
+    k_prefix<D><<<grid, kPreThreads, L::kTotal, stream>>>(a, tk, tv);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
-                          float scale, cudaStream_t stream) {
+cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const void* k_cache, const void* v_cache,
+                          const CUtensorMap& tk, const CUtensorMap& tv, float scale, cudaStream_t stream) {
     const int n = P->hdr.n_prefix_items;
     if (n == 0) return cudaSuccess;
     PrefixArgs a;
     a.items = P->prefix_items;
+    a.n_items = n;
     a.bt = P->bt;
     a.members = P->members;
     a.g_moff = P->g_moff;
@@ -355,13 +512,16 @@ cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const CUtensorMap&
     a.num_blocks = P->num_blocks;
     a.Hq = P->Hq;
     a.G = P->G;
+    a.Hkv = P->Hkv;
     a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k_cache = static_cast<const uint8_t*>(k_cache);
+    a.v_cache = static_cast<const uint8_t*>(v_cache);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.part_o = P->part_o;
     a.part_lse = P->part_lse;
     a.err = P->dev_status;
-    if (P->D == 128) return launch_prefix_t<128>(a, tk, tv, n, stream);
-    return launch_prefix_t<64>(a, tk, tv, n, stream);
+    if (P->D == 128) return launch_prefix_t<128>(a, tk, tv, stream);
+    return launch_prefix_t<64>(a, tk, tv, stream);
 }
 
 }  // namespace fca

@@ -6,18 +6,24 @@
 // is measured against (standard attention, which reads every shared block
 // once per request, "Overview").
 //
-// One CTA per work item = (request, KV head, token chunk).  Warp 0 streams
-// the chunk's paged blocks into a ring of shared-memory slots with TMA
-// (one 16-token x head_dim tile of K and one of V per slot, 128-byte
-// swizzle so that the consumers' strided reads are bank-conflict free).
-// Warps 1-4 take slots round-robin; each keeps its own online-softmax state
-// for the G query heads of the KV head:
-//   - QK: lane = (token t, half of the query rows); full-length dot products
-//     against the pre-scaled fp32 queries in shared memory; softmax maxima and
-//     sums by warp shuffles over the 16 token lanes;
-//   - PV: lane = head_dim slice; probabilities broadcast from shared memory.
-// The four warp states are merged once at the end and written as G partial
-// rows (normalised o, natural-log lse) for the merge pass.
+// Work item = (request, KV head, token chunk); one warp owns one item at a
+// time and keeps everything to itself, so warps never wait for each other:
+//   - its lane 0 streams the chunk's paged 16-token blocks (K and V tiles of
+//     one head, 128-byte swizzle) into the warp's own ring of kSlots
+//     shared-memory slots with TMA, refilling a slot as soon as the warp has
+//     consumed it;
+//   - the G query heads that share the KV head are the N side of warp MMAs
+//     (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the block's 16
+//     tokens on the M side: S^T = K Q^T, then O^T += V^T P^T.  Each lane
+//     holds two query columns, so the online softmax (column max over the
+//     block by three shuffles, per-lane running sums) and the O rescale stay
+//     in registers; P^T reaches the second MMA through movmatrix;
+//   - at the end of the chunk it writes G partial rows (normalised o,
+//     natural-log lse) for the merge pass.
+// Items are taken longest first from a global counter; the last warp out
+// resets the counter for the next launch.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 
 #include "fca_device.cuh"
@@ -27,255 +33,247 @@ namespace fca {
 
 namespace {
 
-constexpr int kSufSlots = 8;
-constexpr int kSufThreads = 160;
+constexpr int kSufWarps = 8;
 
 struct SuffixArgs {
     const SuffixItem* items;
+    int32_t n_items;
     const int32_t* bt;
-    int32_t max_blocks, num_blocks, Hq, G;
+    int32_t max_blocks, Hq, G;
     const __nv_bfloat16* q;
-    float q_scale;            // scale * log2(e)
+    float scale_log2;
     float* part_o;
     float* part_lse;
     int32_t* err;
+    int32_t* sched;           // [0] next item, [1] warps done
 };
 
-template <int D, int GM>
+template <int D>
 struct SufLayout {
-    static constexpr int kHalves = D / 64;
-    static constexpr int kTile = kHalves * 16 * 128;          // one 16-token K (or V) tile
+    static constexpr int kSlots = D == 128 ? 3 : 6;
+    static constexpr int kTile = (D / 64) * 16 * 128;     // one 16-token tile of K (or V), bytes
     static constexpr int kSlot = 2 * kTile;
-    static constexpr int kRing = kSufSlots * kSlot;
-    static constexpr int kQ = GM * D * 4;                     // fp32 queries
-    static constexpr int kP = 4 * (16 * GM + GM) * 4;         // per-warp p[16][GM] + alpha[GM]
-    static constexpr int kComb = 4 * GM * (D + 2) * 4;        // per-warp o, m, l
-    static constexpr int kBars = 2 * kSufSlots * 8 + 16;
-    static constexpr int kTotal = kRing + kQ + kP + kComb + kBars + 1024;   // + alignment slack
+    static constexpr int kWarpRing = kSlots * kSlot;
+    static constexpr int kBars = kSufWarps * kSlots * 8;
+    static constexpr int kTotal = kSufWarps * kWarpRing + kBars + 1024;
 };
 
-template <int D, int GM>
-__global__ void __launch_bounds__(kSufThreads) k_suffix(SuffixArgs a, const __grid_constant__ CUtensorMap tmK,
-                                                        const __grid_constant__ CUtensorMap tmV) {
-    using L = SufLayout<D, GM>;
-    constexpr int RPL = GM / 2;     // query rows per lane (two row halves)
-    constexpr int DPL = D / 32;     // head_dim elements per lane in PV
+// Address of the 16-byte chunk holding (token, element e..e+7) of a tile laid
+// out by TMA with 128-byte swizzle: 64-element halves of 16 rows x 128 B.
+__device__ __forceinline__ uint32_t tile_chunk(uint32_t tile, int tok, int e) {
+    return tile + (e >> 6) * 2048 + tok * 128 + ((((e & 63) >> 3) ^ (tok & 7)) << 4);
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kSufWarps * 32, 1)
+    k_suffix(SuffixArgs a, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+    using L = SufLayout<D>;
+    constexpr int KS = D / 16;        // k-steps of Q K^T, m-tiles of V^T P^T
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* ring = smem;
-    float* qs = reinterpret_cast<float*>(smem + L::kRing);
-    float* ps = reinterpret_cast<float*>(smem + L::kRing + L::kQ);
-    float* comb = reinterpret_cast<float*>(smem + L::kRing + L::kQ + L::kP);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kRing + L::kQ + L::kP + L::kComb);
-    uint64_t* empty = full + kSufSlots;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kSufSlots);
-
-    const SuffixItem it = a.items[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int32_t blk0 = it.tok0 / kBlockSize;
-    const int32_t nblk = (it.tok1 + kBlockSize - 1) / kBlockSize - blk0;
-    const int32_t* row = a.bt + (int64_t)it.request * a.max_blocks;
+    const int g8 = lane >> 2, tig = lane & 3;
+    uint8_t* ring = smem + warp * L::kWarpRing;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSufWarps * L::kWarpRing) + warp * L::kSlots;
+    const uint32_t ring_u32 = dev::smem_u32(ring);
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kSufSlots; ++s) {
-            dev::mbar_init(&full[s], 1);
-            dev::mbar_init(&empty[s], 1);
-        }
-        *abort_flag = 0;
+    if (lane == 0) {
+        for (int s = 0; s < L::kSlots; ++s) dev::mbar_init(&full[s], 1);
         dev::fence_mbarrier_init();
+        dev::tma_prefetch_desc(&tmK);
+        dev::tma_prefetch_desc(&tmV);
     }
-    __syncthreads();
+    __syncwarp();
+    volatile int no_abort = 0;
+    uint32_t uses = 0;        // blocks this warp has pushed through its ring so far
+    bool failed = false;
 
-    if (warp == 0) {
-        // ---------------- producer
-        if (lane == 0) {
-            dev::tma_prefetch_desc(&tmK);
-            dev::tma_prefetch_desc(&tmV);
-            int32_t issued = 0;
-            for (int32_t j = 0; j < nblk; ++j) {
-                const int s = j % kSufSlots;
-                if (j >= kSufSlots &&
-                    !dev::mbar_wait(&empty[s], ((j / kSufSlots) - 1) & 1, abort_flag, a.err))
-                    break;
-                const int32_t phys = row[blk0 + j];
-                uint8_t* kdst = ring + s * L::kSlot;
-                uint8_t* vdst = kdst + L::kTile;
-                dev::mbar_arrive_expect_tx(&full[s], 2 * L::kTile);
+    while (!failed) {
+        int32_t idx = 0;
+        if (lane == 0) idx = atomicAdd(&a.sched[0], 1);
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+        if (idx >= a.n_items) break;
+        const SuffixItem it = a.items[idx];
+        const int32_t blk0 = it.tok0 / kBlockSize;
+        const int32_t nblk = (it.tok1 + kBlockSize - 1) / kBlockSize - blk0;
+        const int32_t* row = a.bt + (int64_t)it.request * a.max_blocks + blk0;
+
+        auto issue = [&](int32_t j) {   // lane 0: block j of the item into its slot
+            const uint32_t u = uses + j;
+            const int s = u % L::kSlots;
+            const int32_t trow = row[j] * kBlockSize;
+            uint8_t* kdst = ring + s * L::kSlot;
+            dev::fence_proxy_async_smem();
+            dev::mbar_arrive_expect_tx(&full[s], L::kSlot);
 #pragma unroll
-                for (int hf = 0; hf < L::kHalves; ++hf) {
-                    dev::tma_load_3d(kdst + hf * 2048, &tmK, &full[s], hf * 64, it.head, phys * kBlockSize);
-                    dev::tma_load_3d(vdst + hf * 2048, &tmV, &full[s], hf * 64, it.head, phys * kBlockSize);
-                }
-                ++issued;
+            for (int hf = 0; hf < D / 64; ++hf) {
+                dev::tma_load_3d(kdst + hf * 2048, &tmK, &full[s], hf * 64, it.head, trow);
+                dev::tma_load_3d(kdst + L::kTile + hf * 2048, &tmV, &full[s], hf * 64, it.head, trow);
             }
-            // never leave with copies in flight
-            for (int32_t j = issued - 1; j >= 0 && j >= issued - kSufSlots; --j) {
-                volatile int never = 0;
-                dev::mbar_wait(&full[j % kSufSlots], (j / kSufSlots) & 1, &never, a.err);
+        };
+        if (lane == 0)
+            for (int32_t j = 0; j < nblk && j < L::kSlots; ++j) issue(j);
+
+        // Q^T fragments (B operand): column n = query head nt * 8 + g8,
+        // rows k = head_dim pairs 16 ks + 2 tig (+8).  Heads past G are zero.
+        uint32_t qb[NT][KS][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int qh = nt * 8 + g8;
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+                a.q + ((int64_t)it.request * a.Hq + it.head * a.G + (qh < a.G ? qh : 0)) * D);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                qb[nt][ks][0] = qh < a.G ? __ldg(qrow + ks * 8 + tig) : 0u;
+                qb[nt][ks][1] = qh < a.G ? __ldg(qrow + ks * 8 + 4 + tig) : 0u;
             }
         }
-        __syncwarp();
-    } else {
-        // ---------------- consumers
-        const int cw = warp - 1;
-        const int ctid = threadIdx.x - 32;
-        // queries, pre-scaled into the log2 domain; padded rows are zero
-        for (int i = ctid; i < GM * D; i += 128) {
-            const int g = i / D, d = i % D;
-            float v = 0.f;
-            if (g < a.G)
-                v = __bfloat162float(a.q[((int64_t)it.request * a.Hq + it.head * a.G + g) * D + d]) * a.q_scale;
-            qs[i] = v;
-        }
-        dev::named_barrier_sync(1, 128);
 
-        const int t = lane & 15, hr = lane >> 4;
-        float m_run[RPL], l_run[RPL];
+        float m_run[NT][2], l_run[NT][2];
+        float o[NT][KS][4];
 #pragma unroll
-        for (int j = 0; j < RPL; ++j) {
-            m_run[j] = -INFINITY;
-            l_run[j] = 0.f;
+        for (int nt = 0; nt < NT; ++nt) {
+            m_run[nt][0] = m_run[nt][1] = -INFINITY;
+            l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
         }
-        float o[GM][DPL];
-#pragma unroll
-        for (int g = 0; g < GM; ++g)
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) o[g][e] = 0.f;
-        float* pw = ps + cw * (16 * GM + GM);     // this warp's p[16][GM], alpha[GM]
-        float* aw = pw + 16 * GM;
 
-        for (int32_t j = cw; j < nblk; j += 4) {
-            const int s = j % kSufSlots;
-            if (!dev::mbar_wait(&full[s], (j / kSufSlots) & 1, abort_flag, a.err)) break;
-            const uint8_t* kt = ring + s * L::kSlot;
-            const uint8_t* vt = kt + L::kTile;
-            const int32_t tok = (blk0 + j) * kBlockSize + t;
+        for (int32_t j = 0; j < nblk; ++j) {
+            const uint32_t u = uses + j;
+            const int s = u % L::kSlots;
+            const bool got = dev::mbar_wait(&full[s], (u / L::kSlots) & 1, &no_abort, a.err);
+            if (!__all_sync(0xffffffffu, got)) { failed = true; break; }
+            const uint32_t kt = ring_u32 + s * L::kSlot, vt = kt + L::kTile;
             const int32_t nvalid = min(kBlockSize, it.tok1 - (blk0 + j) * kBlockSize);
-
-            // scores for (token t, rows hr*RPL + jj)
-            float sc[RPL];
-#pragma unroll
-            for (int jj = 0; jj < RPL; ++jj) sc[jj] = 0.f;
-#pragma unroll 4
-            for (int c = 0; c < D / 8; ++c) {
-                const int hf = c >> 3, cc = c & 7;
-                const uint4 kv = *reinterpret_cast<const uint4*>(kt + hf * 2048 + t * 128 + ((cc ^ (t & 7)) << 4));
-                float kf[8];
-                kf[0] = dev::bf16_lo(kv.x); kf[1] = dev::bf16_hi(kv.x);
-                kf[2] = dev::bf16_lo(kv.y); kf[3] = dev::bf16_hi(kv.y);
-                kf[4] = dev::bf16_lo(kv.z); kf[5] = dev::bf16_hi(kv.z);
-                kf[6] = dev::bf16_lo(kv.w); kf[7] = dev::bf16_hi(kv.w);
-#pragma unroll
-                for (int jj = 0; jj < RPL; ++jj) {
-                    const float* qr = qs + (hr * RPL + jj) * D + c * 8;
-                    const float4 q0 = *reinterpret_cast<const float4*>(qr);
-                    const float4 q1 = *reinterpret_cast<const float4*>(qr + 4);
-                    float acc = sc[jj];
-                    acc = fmaf(q0.x, kf[0], acc); acc = fmaf(q0.y, kf[1], acc);
-                    acc = fmaf(q0.z, kf[2], acc); acc = fmaf(q0.w, kf[3], acc);
-                    acc = fmaf(q1.x, kf[4], acc); acc = fmaf(q1.y, kf[5], acc);
-                    acc = fmaf(q1.z, kf[6], acc); acc = fmaf(q1.w, kf[7], acc);
-                    sc[jj] = acc;
+            if (nvalid < kBlockSize) {
+                // rows past the sequence may hold anything: P is zero there, but
+                // 0 * NaN is not, so clear those V rows before the second MMA
+                uint8_t* vrow = ring + s * L::kSlot + L::kTile;
+                for (int c = lane; c < (kBlockSize - nvalid) * (D / 8); c += 32) {
+                    const int tok = nvalid + c / (D / 8), e = (c % (D / 8)) * 8;
+                    *reinterpret_cast<uint4*>(vrow + (e >> 6) * 2048 + tok * 128 + (e & 63) * 2) =
+                        make_uint4(0, 0, 0, 0);
                 }
+                __syncwarp();
             }
-            const bool valid = tok < it.tok1;
+
+            // S^T = K Q^T: lane holds tokens g8, g8 + 8 x query columns 2 tig, 2 tig + 1
+            float sc[NT][4];
 #pragma unroll
-            for (int jj = 0; jj < RPL; ++jj) {
-                float x = valid ? sc[jj] : -INFINITY;
-                float mx = x;
+            for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
-                for (int off = 1; off < 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                const float m_new = fmaxf(m_run[jj], mx);
-                const float alpha = exp2f(m_run[jj] - m_new);
-                const float p = valid ? exp2f(x - m_new) : 0.f;
-                float ps_sum = p;
+            for (int ks = 0; ks < KS; ++ks) {
+                const int mi = lane >> 3, rr = lane & 7;
+                uint32_t a0, a1, a2, a3;
+                dev::ldsm_x4(tile_chunk(kt, rr + 8 * (mi & 1), ks * 16 + 8 * (mi >> 1)), a0, a1, a2, a3);
 #pragma unroll
-                for (int off = 1; off < 16; off <<= 1) ps_sum += __shfl_xor_sync(0xffffffffu, ps_sum, off);
-                l_run[jj] = l_run[jj] * alpha + ps_sum;
-                m_run[jj] = m_new;
-                pw[t * GM + hr * RPL + jj] = p;
-                if (t == 0) aw[hr * RPL + jj] = alpha;
+                for (int nt = 0; nt < NT; ++nt) dev::mma_bf16_16816(sc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+            }
+
+            uint32_t pb[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float x[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int tok = g8 + (i >> 1) * 8;
+                    x[i] = tok < nvalid ? sc[nt][i] * a.scale_log2 : -INFINITY;
+                }
+                float alpha[2], p[4];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    float mx = fmaxf(x[c], x[c + 2]);
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    const float m_new = fmaxf(m_run[nt][c], mx);
+                    alpha[c] = exp2f(m_run[nt][c] - m_new);
+                    m_run[nt][c] = m_new;
+                    p[c] = exp2f(x[c] - m_new);
+                    p[c + 2] = exp2f(x[c + 2] - m_new);
+                    l_run[nt][c] = l_run[nt][c] * alpha[c] + p[c] + p[c + 2];
+                }
+#pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                    o[nt][mt][0] *= alpha[0];
+                    o[nt][mt][1] *= alpha[1];
+                    o[nt][mt][2] *= alpha[0];
+                    o[nt][mt][3] *= alpha[1];
+                }
+                // P^T as the B operand: transpose the two 8x8 token blocks
+                pb[nt][0] = dev::movmatrix_trans(dev::pack_bf16x2(p[0], p[1]));
+                pb[nt][1] = dev::movmatrix_trans(dev::pack_bf16x2(p[2], p[3]));
+            }
+
+            // O^T += V^T P^T: m-tile mt covers head_dim rows 16 mt .. 16 mt + 15
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                const int mi = lane >> 3, rr = lane & 7;
+                uint32_t a0, a1, a2, a3;
+                dev::ldsm_x4_trans(tile_chunk(vt, rr + 8 * (mi >> 1), mt * 16 + 8 * (mi & 1)), a0, a1, a2, a3);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) dev::mma_bf16_16816(o[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
             }
             __syncwarp();
-            // o = o * alpha + sum_t p_t v_t over this lane's head_dim slice
-#pragma unroll
-            for (int g = 0; g < GM; ++g) {
-                const float al = aw[g];
-#pragma unroll
-                for (int e = 0; e < DPL; ++e) o[g][e] *= al;
-            }
-            const int e0 = lane * DPL;                // first element of the slice
-            const int hf = e0 >> 6, byte_in_half = (e0 & 63) * 2;
-            for (int tt = 0; tt < nvalid; ++tt) {
-                const uint8_t* vrow = vt + hf * 2048 + tt * 128;
-                const int chunk = byte_in_half >> 4, within = byte_in_half & 15;
-                const uint8_t* vp = vrow + ((chunk ^ (tt & 7)) << 4) + within;
-                float vf[DPL];
-                if constexpr (DPL == 4) {
-                    const uint2 vv = *reinterpret_cast<const uint2*>(vp);
-                    vf[0] = dev::bf16_lo(vv.x); vf[1] = dev::bf16_hi(vv.x);
-                    vf[2] = dev::bf16_lo(vv.y); vf[3] = dev::bf16_hi(vv.y);
-                } else {
-                    const uint32_t vv = *reinterpret_cast<const uint32_t*>(vp);
-                    vf[0] = dev::bf16_lo(vv); vf[1] = dev::bf16_hi(vv);
-                }
-                const float* prow = pw + tt * GM;
-#pragma unroll
-                for (int g = 0; g < GM; ++g) {
-                    const float p = prow[g];
-#pragma unroll
-                    for (int e = 0; e < DPL; ++e) o[g][e] = fmaf(p, vf[e], o[g][e]);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) dev::mbar_arrive(&empty[s]);
+            if (lane == 0 && j + L::kSlots < nblk) issue(j + L::kSlots);
         }
+        uses += nblk;
+        if (failed) break;
 
-        // ---------------- merge the four warp states, write G partial rows
-        float* cm = comb;                       // [4][GM] m
-        float* cl = comb + 4 * GM;              // [4][GM] l
-        float* co = comb + 8 * GM;              // [4][GM][D] o
-        if (t == 0) {
+        // column sums over the 8 lanes that share a column, then the partial rows
 #pragma unroll
-            for (int jj = 0; jj < RPL; ++jj) {
-                cm[cw * GM + hr * RPL + jj] = m_run[jj];
-                cl[cw * GM + hr * RPL + jj] = l_run[jj];
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float l = l_run[nt][c];
+                l += __shfl_xor_sync(0xffffffffu, l, 4);
+                l += __shfl_xor_sync(0xffffffffu, l, 8);
+                l += __shfl_xor_sync(0xffffffffu, l, 16);
+                const int qh = nt * 8 + 2 * tig + c;
+                if (qh >= a.G) continue;
+                const float inv = 1.f / l;
+                float* dst = a.part_o + ((int64_t)it.part_row0 + qh) * D;
+#pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                    dst[mt * 16 + g8] = o[nt][mt][c] * inv;
+                    dst[mt * 16 + g8 + 8] = o[nt][mt][c + 2] * inv;
+                }
+                if (g8 == 0) a.part_lse[it.part_row0 + qh] = (m_run[nt][c] + log2f(l)) * 0.69314718055994531f;
             }
         }
-#pragma unroll
-        for (int g = 0; g < GM; ++g)
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) co[(cw * GM + g) * D + lane * DPL + e] = o[g][e];
-        dev::named_barrier_sync(1, 128);
-        for (int i = ctid; i < a.G * D; i += 128) {
-            const int g = i / D, d = i % D;
-            float m = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) m = fmaxf(m, cm[w * GM + g]);
-            float l = 0.f, acc = 0.f;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float mw = cm[w * GM + g];
-                if (mw == -INFINITY) continue;
-                const float sc = exp2f(mw - m);
-                l += cl[w * GM + g] * sc;
-                acc += co[(w * GM + g) * D + d] * sc;
-            }
-            const int64_t prow = it.part_row0 + g;
-            a.part_o[prow * D + d] = acc / l;
-            if (d == 0) a.part_lse[prow] = (m + log2f(l)) * 0.69314718055994531f;
+    }
+
+    // never leave with copies in flight (only after a failed wait)
+    if (failed && lane == 0)
+        for (int s = 0; s < L::kSlots; ++s) {
+            volatile int never = 0;
+            dev::mbar_wait(&full[s], 0, &never, a.err);
+            dev::mbar_wait(&full[s], 1, &never, a.err);
+        }
+    // the last warp to finish resets the item counter for the next launch
+    if (lane == 0) {
+        __threadfence();
+        const int32_t done = atomicAdd(&a.sched[1], 1);
+        if (done == (int32_t)(gridDim.x * kSufWarps) - 1) {
+            a.sched[0] = 0;
+            a.sched[1] = 0;
+            __threadfence();
         }
     }
 }
 
-template <int D, int GM>
-cudaError_t launch_suffix_t(const fca_plan_s* P, const SuffixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                            int n_items, cudaStream_t stream) {
-    using L = SufLayout<D, GM>;
-    cudaError_t e = cudaFuncSetAttribute(k_suffix<D, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
+template <int D, int NT>
+cudaError_t launch_t(const SuffixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
+    using L = SufLayout<D>;
+    cudaError_t e = cudaFuncSetAttribute(k_suffix<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
     if (e != cudaSuccess) return e;
-    k_suffix<D, GM><<<n_items, kSufThreads, L::kTotal, stream>>>(a, tk, tv);
-    (void)P;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int warps_needed = (a.n_items + 1) / 1;
+    const int grid = std::max(1, std::min(sms, (warps_needed + kSufWarps - 1) / kSufWarps));
+    k_suffix<D, NT><<<grid, kSufWarps * 32, L::kTotal, stream>>>(a, tk, tv);
     return cudaGetLastError();
 }
 
@@ -287,27 +285,20 @@ cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap&
     if (n == 0) return cudaSuccess;
     SuffixArgs a;
     a.items = P->suffix_items;
+    a.n_items = n;
     a.bt = P->bt;
     a.max_blocks = P->max_blocks;
-    a.num_blocks = P->num_blocks;
     a.Hq = P->Hq;
     a.G = P->G;
     a.q = static_cast<const __nv_bfloat16*>(q);
-    a.q_scale = scale * 1.4426950408889634f;
+    a.scale_log2 = scale * 1.4426950408889634f;
     a.part_o = P->part_o;
     a.part_lse = P->part_lse;
     a.err = P->dev_status;
-    const int G = P->G;
-    if (P->D == 128) {
-        if (G <= 2) return launch_suffix_t<128, 2>(P, a, tk, tv, n, stream);
-        if (G <= 4) return launch_suffix_t<128, 4>(P, a, tk, tv, n, stream);
-        if (G <= 8) return launch_suffix_t<128, 8>(P, a, tk, tv, n, stream);
-        return launch_suffix_t<128, 16>(P, a, tk, tv, n, stream);
-    }
-    if (G <= 2) return launch_suffix_t<64, 2>(P, a, tk, tv, n, stream);
-    if (G <= 4) return launch_suffix_t<64, 4>(P, a, tk, tv, n, stream);
-    if (G <= 8) return launch_suffix_t<64, 8>(P, a, tk, tv, n, stream);
-    return launch_suffix_t<64, 16>(P, a, tk, tv, n, stream);
+    a.sched = P->sched;
+    const bool two = P->G > 8;
+    if (P->D == 128) return two ? launch_t<128, 2>(a, tk, tv, stream) : launch_t<128, 1>(a, tk, tv, stream);
+    return two ? launch_t<64, 2>(a, tk, tv, stream) : launch_t<64, 1>(a, tk, tv, stream);
 }
 
 }  // namespace fca

@@ -161,6 +161,54 @@ def test_lse_optional():
     assert_close(o, None, o_ref, None, "no lse")
 
 
+def growing_keys_workload(seed=0):
+    """One 16-request group over a 1024-token prompt whose key norms grow
+    with the logical position, so the running maximum keeps rising from stage
+    to stage (exercises the grouped pass's rescaling of its accumulator)."""
+    rng = np.random.default_rng(seed)
+    reqs = [[("p", 1024), (None, int(rng.integers(1, 200)))] for _ in range(16)]
+    w = fca_workloads.fill("growing", reqs, Hq=16, Hkv=2, D=128, seed=seed, rng=rng)
+    k = (w.k_cache.astype(np.uint32) << 16).view(np.float32).copy()
+    done = np.zeros(w.num_blocks, bool)
+    for r in range(w.R):
+        nblk = (int(w.seq_lens[r]) + 15) // 16
+        for j in range(nblk):
+            b = w.block_tables[r, j]
+            if not done[b]:
+                k[b] *= 0.25 * (1 + j)
+                done[b] = True
+    u = k.view(np.uint32)
+    w.k_cache = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    # the softmax ends up peaked on single tokens; keep |o| < 2, where half a
+    # bf16 ulp of the output (3.9e-3) stays inside the 1e-2 bound
+    v = (w.v_cache.astype(np.uint32) << 16).view(np.float32) * 0.4
+    u = v.view(np.uint32)
+    w.v_cache = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    return w
+
+
+@pytest.mark.parametrize("split", [0, 256])
+def test_prefix_rescale_path(split):
+    w = growing_keys_workload()
+    o, l, exp, _ = run(w, split_tokens=split)
+    assert len(exp["a"]) == 1
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(o, l, o_ref, l_ref, f"growing keys split {split}")
+
+
+def test_many_items_per_cta():
+    # far more grouped-pass items than SMs: every CTA walks several items
+    for seed in (1, 2):
+        w = fca_workloads.make("llama8b", seed=seed, prompts=4)
+        o, l, _, st = run(w, split_tokens=64)
+        assert st["prefix_items"] > 4 * 148
+        pairs = sampled_pairs(w, 64, seed)
+        o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens,
+                                              w.scale, pairs=pairs)
+        sel = (pairs[:, 0], pairs[:, 1])
+        assert_close(o[sel], l[sel], o_ref, l_ref, "many items")
+
+
 # --------------------------------------------------------------- full-size configurations
 
 def sampled_pairs(w, n, seed=0):
