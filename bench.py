@@ -8,8 +8,11 @@ A step is one pass of the whole hot path -- grouped prefix pass, per-request
 pass, log-sum-exp merge -- over the configuration's synthetic batch, with the
 plan built beforehand (plan time is reported separately).  Inputs are
 resident in HBM; L2 is flushed (256 MiB write) before every timed step.
-Every step is timed on the device with CUDA events on the launching stream,
-per pass; ms_per_step is the mean over the K timed steps (max over ranks).
+Every step is one fca_decode call (the two passes run side by side on
+disjoint SMs, then the merge), timed on the device with CUDA events on the
+launching stream; ms_per_step is the mean over the K timed steps (max over
+ranks).  The roofline times each pass alone on every SM through its own
+entry point, in a second loop after the timed region.
 
 value = unique KV bytes processed by all ranks per step / ms_per_step, in
 GB/s (each shared block counted once).  Under torchrun every rank decodes its
@@ -286,6 +289,23 @@ def fca_arm(args):
                                                        split_tokens=args.split)
 
     def run_steps(p, n, timed):
+        """n whole decode steps (fca_decode: both passes side by side, then the
+        merge), each bracketed by events on the launching stream."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            ev[i][0].record(stream)
+            fca.fca_decode(q, k, v, p, out, lse, w.scale, stream)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        if not timed:
+            return None
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    def run_passes(p, n, timed):
+        """n steps with the three passes launched one after another through
+        their own entry points, each pass on every SM and bracketed by events
+        on the launching stream: the per-kernel durations of the roofline."""
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
         for i in range(n):
             flush.zero_()
@@ -316,22 +336,28 @@ def fca_arm(args):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    fca_t = run_steps(plan, args.steps, True)
+    step_ms = run_steps(plan, args.steps, True)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop() if sampler else None
     barrier()
     assert fca.fca_check_device_status(plan, stream) == 0
-    step_ms = max_over_ranks(fca_t["step"])
+    step_ms = max_over_ranks(step_ms)
     n_launch = (1 if (st["prefix_items"] > 0) else 0) + (1 if st["suffix_items"] > 0 else 0) + 1
+
+    # ---- the passes one at a time (per-kernel roofline)
+    run_passes(plan, args.warmup, False)
+    barrier()
+    fca_t = run_passes(plan, args.steps, True)
+    barrier()
+    assert fca.fca_check_device_status(plan, stream) == 0
 
     # ---- flat paged decode of the same batch
     flat_ms = None
     if flat_plan is not None:
         run_steps(flat_plan, args.warmup, False)
         barrier()
-        flat_t = run_steps(flat_plan, args.steps, True)
+        flat_ms = max_over_ranks(run_steps(flat_plan, args.steps, True))
         barrier()
-        flat_ms = max_over_ranks(flat_t["step"])
         assert fca.fca_check_device_status(flat_plan, stream) == 0
 
     # ---- end to end through the public API with host buffers
@@ -382,6 +408,7 @@ def fca_arm(args):
 
     # dominant kernel and its roofline
     pass_ms = {key: max_over_ranks(fca_t[key]) for key in ("prefix", "suffix", "merge")}
+    serial_ms = max_over_ranks(fca_t["step"])
     dominant = max(pass_ms, key=pass_ms.get)
     alg_bytes = {"prefix": st["prefix_kv_bytes"], "suffix": st["suffix_kv_bytes"],
                  "merge": st["num_partials"] * (w.D + 1) * 4 + w.R * w.Hq * (w.D * 2 + 4)}
@@ -410,6 +437,7 @@ def fca_arm(args):
             "pct_of_peak": 100.0 * value / (peak * world), "peak_gbs": peak, "peak_kind": peak_kind,
             "plan_ms": plan_ms,
             "passes_us": {key: val * 1e3 for key, val in pass_ms.items()},
+            "serial_passes_us_per_step": serial_ms * 1e3,
             "flat_us_per_step": flat_ms * 1e3 if flat_ms else None,
             "speedup_vs_flat": (flat_ms / step_ms) if flat_ms else None,
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,

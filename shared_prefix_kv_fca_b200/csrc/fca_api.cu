@@ -1,6 +1,8 @@
 // C ABI of libfca_b200 (declared in include/fca.h): argument checks, plan
 // lifetime, TMA descriptors and the launch order of one decode step.
+#include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -9,10 +11,10 @@
 
 namespace fca {
 fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cudaStream_t stream, fca_plan_s* P);
-cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const void* k_cache, const void* v_cache,
-                          const CUtensorMap& tk, const CUtensorMap& tv, float scale, cudaStream_t stream);
+cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
+                          float scale, int max_ctas, cudaStream_t stream);
 cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
-                          float scale, cudaStream_t stream);
+                          float scale, int max_ctas, cudaStream_t stream);
 cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, cudaStream_t stream);
 
 namespace {
@@ -81,6 +83,9 @@ fca_status fca_plan_destroy(fca_plan_t plan) {
     if (!plan) return FCA_OK;
     cudaDeviceSynchronize();
     for (void* p : plan->dev_allocs) cudaFree(p);
+    if (plan->aux_stream) cudaStreamDestroy(plan->aux_stream);
+    if (plan->ev_fork) cudaEventDestroy(plan->ev_fork);
+    if (plan->ev_join) cudaEventDestroy(plan->ev_join);
     (void)cudaGetLastError();
     delete plan;
     return FCA_OK;
@@ -124,6 +129,22 @@ fca_status fca_plan(const int32_t* block_tables, int32_t max_blocks, const int32
     return FCA_OK;
 }
 
+// SMs given to the grouped pass when it runs beside the per-request pass.
+// Rates per SM measured on B200 with both passes running: about 12.5 GB/s
+// for the grouped pass (its per-head reads use an eighth of each DRAM row, so
+// it is bound by row activations rather than by bandwidth) and 49 GB/s for
+// the per-request pass.  The grouped pass gets 0.9 of the SMs that would make
+// both finish together; both passes take their items longest first from a
+// queue, and a sweep over the split on four workloads put this within 1-8%
+// of the best fixed split.  Each pass is launched on its own SMs: run on
+// every SM, the per-request pass shares SMs with the grouped one and slows it.
+static int prefix_share(const fca_plan_s* P, int sms) {
+    const double tp = (double)P->hdr.prefix_tok_sum / 12.5;
+    const double ts = (double)P->hdr.suffix_tok_sum / 49.0;
+    const int n = (int)(0.9 * sms * tp / (tp + ts) + 0.5);
+    return std::max(1, std::min(sms - 1, n));
+}
+
 static fca_status decode_impl(const void* q, const void* k_cache, const void* v_cache, fca_plan_t plan, void* out,
                               float* lse, float scale, void* stream) {
     if (!plan || !q || !k_cache || !v_cache || !out) return FCA_ERR_INVALID_ARG;
@@ -135,9 +156,34 @@ static fca_status decode_impl(const void* q, const void* k_cache, const void* v_
     if (!make_cache_map(&tk, k_cache, plan->num_blocks, plan->Hkv, plan->D) ||
         !make_cache_map(&tv, v_cache, plan->num_blocks, plan->Hkv, plan->D))
         return FCA_ERR_CUDA;
-    if (!plan->flat && plan->hdr.n_prefix_items > 0 && note_cuda(launch_prefix(plan, q, k_cache, v_cache, tk, tv, scale, s)) != cudaSuccess)
-        return FCA_ERR_CUDA;
-    if (note_cuda(launch_suffix(plan, q, tk, tv, scale, s)) != cudaSuccess) return FCA_ERR_CUDA;
+    const bool grouped = !plan->flat && plan->hdr.n_prefix_items > 0;
+    if (grouped && plan->hdr.n_suffix_items > 0) {
+        // The two passes are independent: run them side by side on disjoint SMs.
+        if (!plan->aux_stream) {
+            // highest priority, so the grouped pass's CTAs are placed first
+            int lo = 0, hi = 0;
+            cudaDeviceGetStreamPriorityRange(&lo, &hi);
+            if (note_cuda(cudaStreamCreateWithPriority(&plan->aux_stream, cudaStreamNonBlocking, hi)) != cudaSuccess ||
+                note_cuda(cudaEventCreateWithFlags(&plan->ev_fork, cudaEventDisableTiming)) != cudaSuccess ||
+                note_cuda(cudaEventCreateWithFlags(&plan->ev_join, cudaEventDisableTiming)) != cudaSuccess)
+                return FCA_ERR_CUDA;
+        }
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int np = prefix_share(plan, sms);
+        if (note_cuda(cudaEventRecord(plan->ev_fork, s)) != cudaSuccess ||
+            note_cuda(cudaStreamWaitEvent(plan->aux_stream, plan->ev_fork, 0)) != cudaSuccess ||
+            note_cuda(launch_prefix(plan, q, tk, tv, scale, np, plan->aux_stream)) != cudaSuccess ||
+            note_cuda(launch_suffix(plan, q, tk, tv, scale, sms - np, s)) != cudaSuccess ||
+            note_cuda(cudaEventRecord(plan->ev_join, plan->aux_stream)) != cudaSuccess ||
+            note_cuda(cudaStreamWaitEvent(s, plan->ev_join, 0)) != cudaSuccess)
+            return FCA_ERR_CUDA;
+    } else {
+        if (grouped && note_cuda(launch_prefix(plan, q, tk, tv, scale, 0, s)) != cudaSuccess)
+            return FCA_ERR_CUDA;
+        if (note_cuda(launch_suffix(plan, q, tk, tv, scale, 0, s)) != cudaSuccess) return FCA_ERR_CUDA;
+    }
     if (note_cuda(launch_merge(plan, out, lse, s)) != cudaSuccess) return FCA_ERR_CUDA;
     return FCA_OK;
 }
@@ -158,9 +204,10 @@ static fca_status pass_impl(int pass, const void* q, const void* k_cache, const 
         return FCA_ERR_CUDA;
     if (pass == 0) {
         if (plan->flat || plan->hdr.n_prefix_items == 0) return FCA_OK;
-        return note_cuda(launch_prefix(plan, q, k_cache, v_cache, tk, tv, scale, s)) == cudaSuccess ? FCA_OK : FCA_ERR_CUDA;
+        return note_cuda(launch_prefix(plan, q, tk, tv, scale, 0, s)) == cudaSuccess ? FCA_OK
+                                                                                                   : FCA_ERR_CUDA;
     }
-    return note_cuda(launch_suffix(plan, q, tk, tv, scale, s)) == cudaSuccess ? FCA_OK : FCA_ERR_CUDA;
+    return note_cuda(launch_suffix(plan, q, tk, tv, scale, 0, s)) == cudaSuccess ? FCA_OK : FCA_ERR_CUDA;
 }
 
 fca_status fca_prefix_pass(const void* q, const void* k_cache, const void* v_cache, fca_plan_t plan, float scale,

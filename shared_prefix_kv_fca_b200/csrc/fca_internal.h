@@ -108,6 +108,10 @@ struct fca_plan_s {
     float* part_lse = nullptr;       // [n_partials]
     int32_t* dev_status = nullptr;   // device error word
 
+    // side stream and events for running the two passes side by side
+    cudaStream_t aux_stream = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+
     // every cudaMalloc the plan owns (freed by fca_plan_destroy)
     std::vector<void*> dev_allocs;
 };

@@ -58,10 +58,8 @@ struct PrefixArgs {
     const int32_t* bt;
     const int32_t* members;
     const int32_t* g_moff;
-    int32_t max_blocks, num_blocks, Hq, G, Hkv;
+    int32_t max_blocks, num_blocks, Hq, G;
     const __nv_bfloat16* q;
-    const uint8_t* k_cache;   // raw cache bases, for whole-block L2 prefetch
-    const uint8_t* v_cache;
     float scale_log2;
     float* part_o;
     float* part_lse;
@@ -484,13 +482,15 @@ __global__ void __launch_bounds__(kPreThreads, 1)
 }
 
 template <int D>
-cudaError_t launch_prefix_t(const PrefixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
+cudaError_t launch_prefix_t(const PrefixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int max_ctas,
+                            cudaStream_t stream) {
     using L = PreLayout<D>;
     cudaError_t e = cudaFuncSetAttribute(k_prefix<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (max_ctas > 0) sms = std::min(sms, max_ctas);
     const int grid = std::max(1, std::min(sms, a.n_items));
     k_prefix<D><<<grid, kPreThreads, L::kTotal, stream>>>(a, tk, tv);
     return cudaGetLastError();
@@ -498,8 +498,8 @@ cudaError_t launch_prefix_t(const PrefixArgs& a, const CUtensorMap& tk, const CU
 
 }  // namespace
 
-cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const void* k_cache, const void* v_cache,
-                          const CUtensorMap& tk, const CUtensorMap& tv, float scale, cudaStream_t stream) {
+cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
+                          float scale, int max_ctas, cudaStream_t stream) {
     const int n = P->hdr.n_prefix_items;
     if (n == 0) return cudaSuccess;
     PrefixArgs a;
@@ -512,16 +512,13 @@ cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const void* k_cach
     a.num_blocks = P->num_blocks;
     a.Hq = P->Hq;
     a.G = P->G;
-    a.Hkv = P->Hkv;
     a.q = static_cast<const __nv_bfloat16*>(q);
-    a.k_cache = static_cast<const uint8_t*>(k_cache);
-    a.v_cache = static_cast<const uint8_t*>(v_cache);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.part_o = P->part_o;
     a.part_lse = P->part_lse;
     a.err = P->dev_status;
-    if (P->D == 128) return launch_prefix_t<128>(a, tk, tv, stream);
-    return launch_prefix_t<64>(a, tk, tv, stream);
+    if (P->D == 128) return launch_prefix_t<128>(a, tk, tv, max_ctas, stream);
+    return launch_prefix_t<64>(a, tk, tv, max_ctas, stream);
 }
 
 }  // namespace fca

@@ -264,15 +264,16 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
 }
 
 template <int D, int NT>
-cudaError_t launch_t(const SuffixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
+cudaError_t launch_t(const SuffixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int max_ctas,
+                     cudaStream_t stream) {
     using L = SufLayout<D>;
     cudaError_t e = cudaFuncSetAttribute(k_suffix<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int warps_needed = (a.n_items + 1) / 1;
-    const int grid = std::max(1, std::min(sms, (warps_needed + kSufWarps - 1) / kSufWarps));
+    if (max_ctas > 0) sms = std::min(sms, max_ctas);
+    const int grid = std::max(1, std::min(sms, (a.n_items + kSufWarps - 1) / kSufWarps));
     k_suffix<D, NT><<<grid, kSufWarps * 32, L::kTotal, stream>>>(a, tk, tv);
     return cudaGetLastError();
 }
@@ -280,7 +281,7 @@ cudaError_t launch_t(const SuffixArgs& a, const CUtensorMap& tk, const CUtensorM
 }  // namespace
 
 cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
-                          float scale, cudaStream_t stream) {
+                          float scale, int max_ctas, cudaStream_t stream) {
     const int n = P->hdr.n_suffix_items;
     if (n == 0) return cudaSuccess;
     SuffixArgs a;
@@ -297,8 +298,9 @@ cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap&
     a.err = P->dev_status;
     a.sched = P->sched;
     const bool two = P->G > 8;
-    if (P->D == 128) return two ? launch_t<128, 2>(a, tk, tv, stream) : launch_t<128, 1>(a, tk, tv, stream);
-    return two ? launch_t<64, 2>(a, tk, tv, stream) : launch_t<64, 1>(a, tk, tv, stream);
+    if (P->D == 128)
+        return two ? launch_t<128, 2>(a, tk, tv, max_ctas, stream) : launch_t<128, 1>(a, tk, tv, max_ctas, stream);
+    return two ? launch_t<64, 2>(a, tk, tv, max_ctas, stream) : launch_t<64, 1>(a, tk, tv, max_ctas, stream);
 }
 
 }  // namespace fca
