@@ -51,7 +51,8 @@ typedef enum fca_status {
     FCA_ERR_UNSUPPORTED = 3,   /* valid input this build does not handle (e.g. head_dim) */
     FCA_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
     FCA_ERR_OOM = 5,           /* device allocation failed */
-    FCA_ERR_DEVICE_FLAG = 6    /* a kernel reported an internal error (bounded wait ran out) */
+    FCA_ERR_DEVICE_FLAG = 6,   /* a kernel reported an internal error (bounded wait ran out) */
+    FCA_ERR_TOO_LARGE = 7      /* fca_paged_decode_static: the problem exceeds its fixed scratch */
 } fca_status;
 
 /* Opaque plan: the group forest, per-request suffix starts, the work lists of
@@ -113,9 +114,14 @@ fca_status fca_plan(const int32_t *block_tables, int32_t max_blocks, const int32
  *   lse      DEVICE fp32 [num_requests][num_q_heads], or NULL to skip.
  *   scale    multiplier of q.k (normally 1/sqrt(head_dim)).
  *
- * Asynchronous on `stream`; uses the plan's workspace, so decodes that share
- * a plan must be ordered on one stream.  A kernel that detects an internal
- * error records it in the plan; read it with fca_check_device_status.
+ * Asynchronous on `stream`.  When the plan has both grouped and per-request
+ * work, the two passes run side by side on disjoint sets of SMs: the grouped
+ * pass on a high-priority side stream that the plan creates on its first
+ * decode (ordered after the work already queued on `stream` by an event),
+ * the per-request pass on `stream`; the merge waits for both.  Uses the
+ * plan's workspace, so decodes that share a plan must be ordered on one
+ * stream.  A kernel that detects an internal error records it in the plan;
+ * read it with fca_check_device_status.
  */
 fca_status fca_decode(const void *q, const void *k_cache, const void *v_cache, fca_plan_t plan,
                       void *out, float *lse, float scale, void *stream);
@@ -134,9 +140,11 @@ fca_status fca_flat_decode(const void *q, const void *k_cache, const void *v_cac
  * runs them: fca_prefix_pass (grouped pass over shared prefix blocks, no-op
  * for a flat plan or a plan without groups), fca_suffix_pass (per-request
  * pass over own blocks) and fca_merge_pass (log-sum-exp reduction into out
- * and lse).  Running the three in order on one stream is exactly fca_decode;
- * they exist so that each kernel can be timed on its own stream.  The first
- * two write only the plan's partial buffers.  Arguments as fca_decode.
+ * and lse).  Each runs on every SM.  Running the three in order on one
+ * stream gives exactly the result of fca_decode (every work item writes its
+ * own partial rows, whichever SM runs it); they exist so that each kernel can
+ * be timed alone.  The first two write only the plan's partial buffers.
+ * Arguments as fca_decode.
  */
 fca_status fca_prefix_pass(const void *q, const void *k_cache, const void *v_cache, fca_plan_t plan,
                            float scale, void *stream);
@@ -191,6 +199,61 @@ fca_status fca_plan_destroy(fca_plan_t plan);
  * word was non-zero.
  */
 fca_status fca_check_device_status(fca_plan_t plan, void *stream, int32_t *code);
+
+/*
+ * fca_paged_decode_static -- the flat paged decode of fca_flat_decode
+ * (standard split-KV attention of every request over its whole block table,
+ * then the log-sum-exp merge) in one call that allocates nothing.  This entry
+ * has no counterpart in the method's description ("ZoRRo Inference & Forest
+ * Cascade Attention"); it is for callers that cannot allocate device memory
+ * at decode time: an engine whose device memory is all handed out by its own
+ * pool, or code that must not call the CUDA allocator while it records a
+ * stream.  It needs no plan; it does not share prefix blocks.
+ *
+ * Memory: the work list and the partial results live in one fixed device
+ * array of this library, 64 MiB (FCA_STATIC_SCRATCH_BYTES) on each device,
+ * set aside by the CUDA runtime when it loads the library's kernels there.
+ * The call itself makes no cudaMalloc, cudaFree or other allocating call:
+ * it issues one cudaMemsetAsync of 16 bytes and three kernels on `stream`.
+ * The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress), which may load the library's kernels on that
+ * device; make that first call before any stream capture.
+ *
+ * What must start at zero: the array's three work counters, which the call
+ * zeroes itself on `stream` before its kernels; and *dev_status, which the
+ * caller zeroes.
+ *
+ * Concurrency: every call on a device uses the same array.  Calls must be
+ * ordered (one stream, or events between streams); two calls in flight at
+ * once on one device race and both results are undefined.
+ *
+ *   q, k_cache, v_cache, out, lse, scale  as fca_decode.
+ *   block_tables  DEVICE int32 [num_requests][max_blocks], 4-byte aligned.
+ *   seq_lens      DEVICE int32 [num_requests]; each in [1, max_blocks * 16].
+ *   num_blocks    physical blocks in each cache (block size 16).
+ *   dev_status    DEVICE int32, or NULL: the kernels OR error bits into it:
+ *                 1 a bounded wait ran out, 2 a work item failed its range
+ *                 check, 8 a seq_len out of range, 16 a used block id out of
+ *                 [0, num_blocks).  A request with a bad length or id is
+ *                 skipped (its out rows are 0, its lse -inf).  With NULL the
+ *                 bits are dropped.
+ *
+ * Returns FCA_ERR_INVALID_ARG (null or misaligned pointer, bad shape),
+ * FCA_ERR_UNSUPPORTED (head_dim not 64 or 128, more than 16 query heads per
+ * KV head), FCA_ERR_TOO_LARGE when num_requests x num_q_heads partial rows
+ * of one split each, plus the work list, exceed the array (about
+ * num_requests * num_q_heads * (head_dim + 1) * 4 + num_requests *
+ * num_kv_heads * 32 bytes must stay under 64 MiB; e.g. up to 3900 requests
+ * at 32 query heads of head_dim 128), FCA_ERR_CUDA.  num_requests == 0 is a
+ * no-op.  Asynchronous on `stream`.
+ */
+#define FCA_STATIC_SCRATCH_BYTES (64u << 20)
+fca_status fca_paged_decode_static(const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *block_tables, int32_t max_blocks,
+                                   const int32_t *seq_lens, int32_t num_requests, int32_t num_blocks,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                   void *out, float *lse, float scale, int32_t *dev_status,
+                                   void *stream);
 
 /* Text of the last CUDA error a call of this library met on the calling
  * thread ("no error" if none); valid until the next failing call. */

@@ -27,7 +27,7 @@ __all__ = [
     "fca_plan_export", "fca_plan_member_count", "fca_plan_destroy", "fca_check_device_status",
     "fca_status_string", "fca_version", "fca_plan_opts_default", "library_path", "load_library",
     "fca_prefix_pass", "fca_suffix_pass", "fca_merge_pass", "fca_last_cuda_error",
-    "FCA_PLAN_FLAT", "STATUS",
+    "FCA_PLAN_FLAT", "STATUS", "fca_paged_decode_static", "FCA_STATIC_SCRATCH_BYTES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -36,7 +36,8 @@ _lib = None
 
 FCA_PLAN_FLAT = 1
 STATUS = {0: "FCA_OK", 1: "FCA_ERR_INVALID_ARG", 2: "FCA_ERR_BAD_BLOCK_ID", 3: "FCA_ERR_UNSUPPORTED",
-          4: "FCA_ERR_CUDA", 5: "FCA_ERR_OOM", 6: "FCA_ERR_DEVICE_FLAG"}
+          4: "FCA_ERR_CUDA", 5: "FCA_ERR_OOM", 6: "FCA_ERR_DEVICE_FLAG", 7: "FCA_ERR_TOO_LARGE"}
+FCA_STATIC_SCRATCH_BYTES = 64 << 20
 
 
 class FcaError(RuntimeError):
@@ -106,6 +107,9 @@ def load_library():
     lib.fca_plan_destroy.restype = ctypes.c_int
     lib.fca_check_device_status.argtypes = [vp, vp, i32p]
     lib.fca_check_device_status.restype = ctypes.c_int
+    lib.fca_paged_decode_static.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, vp, vp, f32,
+                                            vp, vp]
+    lib.fca_paged_decode_static.restype = ctypes.c_int
     lib.fca_status_string.argtypes = [ctypes.c_int]
     lib.fca_status_string.restype = ctypes.c_char_p
     lib.fca_version.argtypes = []
@@ -195,6 +199,36 @@ def fca_flat_decode(q, k_cache, v_cache, plan: "Plan", out, lse=None, scale=None
                     stream=None) -> None:
     """Flat (non-cascaded) paged decode; plan must be built with flat=True."""
     _decode("fca_flat_decode", q, k_cache, v_cache, plan, out, lse, scale, stream)
+
+
+def fca_paged_decode_static(q, k_cache, v_cache, block_tables, seq_lens, num_blocks: int, out, lse=None,
+                            scale=None, dev_status=None, stream=None) -> None:
+    """Flat paged decode that allocates nothing (no plan; work list and
+    partials in the library's fixed 64 MiB device array).  q/out bf16
+    [R, Hq, D]; caches bf16 [num_blocks, 16, Hkv, D]; block_tables int32
+    [R, max_blocks] and seq_lens int32 [R] CUDA tensors; dev_status an int32
+    CUDA tensor of one element (zeroed by the caller) or None.  Calls on one
+    device must be ordered: they share the array."""
+    lib = load_library()
+    for t, name in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (out, "out")):
+        if not t.is_cuda or str(t.dtype) != "torch.bfloat16" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens")):
+        if not t.is_cuda or str(t.dtype) != "torch.int32" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    if lse is not None and (str(lse.dtype) != "torch.float32" or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 CUDA tensor")
+    if dev_status is not None and (str(dev_status.dtype) != "torch.int32" or dev_status.numel() < 1):
+        raise ValueError("dev_status must be an int32 CUDA tensor of at least one element")
+    R, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rc = lib.fca_paged_decode_static(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                     block_tables.shape[1], _ptr(seq_lens), R, num_blocks, Hq, Hkv, D,
+                                     _ptr(out), _ptr(lse), float(scale), _ptr(dev_status),
+                                     _stream_handle(stream))
+    _check(rc, "fca_paged_decode_static")
 
 
 def fca_prefix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) -> None:

@@ -47,6 +47,8 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+}  // namespace
+
 // Cache [num_blocks * 16 tokens][Hkv][D] bf16 viewed as a 3-D tensor
 // (innermost first: D, Hkv, tokens); box = 64 head-dim elements x 1 head x
 // 16 tokens (one paged block of one head, one 128-byte swizzle atom wide).
@@ -62,9 +64,6 @@ bool make_cache_map(CUtensorMap* map, const void* base, int32_t num_blocks, int3
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-}  // namespace
 }  // namespace fca
 
 using namespace fca;
@@ -317,6 +316,7 @@ const char* fca_status_string(fca_status status) {
         case FCA_ERR_CUDA: return "CUDA error";
         case FCA_ERR_OOM: return "out of device memory";
         case FCA_ERR_DEVICE_FLAG: return "kernel reported an internal error";
+        case FCA_ERR_TOO_LARGE: return "problem larger than the fixed scratch of fca_paged_decode_static";
     }
     return "unknown status";
 }

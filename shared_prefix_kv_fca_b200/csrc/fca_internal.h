@@ -25,6 +25,14 @@ constexpr int32_t kErrWaitTimeout = 1;     // a bounded mbarrier wait ran out
 constexpr int32_t kErrBadItem = 2;         // a work item failed its own range check
 constexpr int32_t kErrPlanInternal = 4;    // a planner consistency check failed (no write done)
 
+// Raised by the work-list kernel of fca_paged_decode_static, which cannot
+// return an error to the host: the request is skipped (out 0, lse -inf).
+constexpr int32_t kErrStaticSeqLen = 8;    // seq_len outside [1, max_blocks * block_size]
+constexpr int32_t kErrStaticBlockId = 16;  // a used table entry outside [0, num_blocks)
+
+// Size of the fixed device array behind fca_paged_decode_static.
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+
 // Planner status bits (read back inside fca_plan).
 constexpr int32_t kPlanBadSeqLen = 1;
 constexpr int32_t kPlanBadBlockId = 2;
@@ -68,6 +76,11 @@ struct PlanHeader {
 
 // Remember e (if it is an error) as the calling thread's last CUDA error.
 cudaError_t note_cuda(cudaError_t e);
+
+// TMA descriptor of a K or V cache [num_blocks * 16][Hkv][D] bf16 (fca_api.cu).
+bool make_cache_map(CUtensorMap* map, const void* base, int32_t num_blocks, int32_t Hkv, int32_t D);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace fca
 

@@ -64,7 +64,10 @@ __device__ __forceinline__ uint32_t tile_chunk(uint32_t tile, int tok, int e) {
     return tile + (e >> 6) * 2048 + tok * 128 + ((((e & 63) >> 3) ^ (tok & 7)) << 4);
 }
 
-template <int D, int NT>
+// kDevCount: the item count is read from sched[2], written on the device by
+// the kernel that built the items (a.n_items is then only the bound the grid
+// was sized for).
+template <int D, int NT, bool kDevCount>
 __global__ void __launch_bounds__(kSufWarps * 32, 1)
     k_suffix(SuffixArgs a, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
     using L = SufLayout<D>;
@@ -85,6 +88,7 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
     }
     __syncwarp();
     volatile int no_abort = 0;
+    const int32_t n_items = kDevCount ? *reinterpret_cast<volatile const int32_t*>(a.sched + 2) : a.n_items;
     uint32_t uses = 0;        // blocks this warp has pushed through its ring so far
     bool failed = false;
 
@@ -92,7 +96,7 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
         int32_t idx = 0;
         if (lane == 0) idx = atomicAdd(&a.sched[0], 1);
         idx = __shfl_sync(0xffffffffu, idx, 0);
-        if (idx >= a.n_items) break;
+        if (idx >= n_items) break;
         const SuffixItem it = a.items[idx];
         const int32_t blk0 = it.tok0 / kBlockSize;
         const int32_t nblk = (it.tok1 + kBlockSize - 1) / kBlockSize - blk0;
@@ -263,30 +267,26 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
     }
 }
 
-template <int D, int NT>
+template <int D, int NT, bool kDevCount = false>
 cudaError_t launch_t(const SuffixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int max_ctas,
                      cudaStream_t stream) {
     using L = SufLayout<D>;
-    cudaError_t e = cudaFuncSetAttribute(k_suffix<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_suffix<D, NT, kDevCount>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (max_ctas > 0) sms = std::min(sms, max_ctas);
     const int grid = std::max(1, std::min(sms, (a.n_items + kSufWarps - 1) / kSufWarps));
-    k_suffix<D, NT><<<grid, kSufWarps * 32, L::kTotal, stream>>>(a, tk, tv);
+    k_suffix<D, NT, kDevCount><<<grid, kSufWarps * 32, L::kTotal, stream>>>(a, tk, tv);
     return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
-                          float scale, int max_ctas, cudaStream_t stream) {
-    const int n = P->hdr.n_suffix_items;
-    if (n == 0) return cudaSuccess;
+SuffixArgs suffix_args(const fca_plan_s* P, const void* q, float scale) {
     SuffixArgs a;
     a.items = P->suffix_items;
-    a.n_items = n;
+    a.n_items = P->hdr.n_suffix_items;
     a.bt = P->bt;
     a.max_blocks = P->max_blocks;
     a.Hq = P->Hq;
@@ -297,10 +297,29 @@ cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap&
     a.part_lse = P->part_lse;
     a.err = P->dev_status;
     a.sched = P->sched;
+    return a;
+}
+
+}  // namespace
+
+cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
+                          float scale, int max_ctas, cudaStream_t stream) {
+    if (P->hdr.n_suffix_items == 0) return cudaSuccess;
+    const SuffixArgs a = suffix_args(P, q, scale);
     const bool two = P->G > 8;
     if (P->D == 128)
         return two ? launch_t<128, 2>(a, tk, tv, max_ctas, stream) : launch_t<128, 1>(a, tk, tv, max_ctas, stream);
     return two ? launch_t<64, 2>(a, tk, tv, max_ctas, stream) : launch_t<64, 1>(a, tk, tv, max_ctas, stream);
+}
+
+cudaError_t launch_suffix_devcount(const fca_plan_s* P, const void* q, const CUtensorMap& tk,
+                                   const CUtensorMap& tv, float scale, cudaStream_t stream) {
+    if (P->hdr.n_suffix_items == 0) return cudaSuccess;
+    const SuffixArgs a = suffix_args(P, q, scale);
+    const bool two = P->G > 8;
+    if (P->D == 128)
+        return two ? launch_t<128, 2, true>(a, tk, tv, 0, stream) : launch_t<128, 1, true>(a, tk, tv, 0, stream);
+    return two ? launch_t<64, 2, true>(a, tk, tv, 0, stream) : launch_t<64, 1, true>(a, tk, tv, 0, stream);
 }
 
 }  // namespace fca
