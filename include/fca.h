@@ -93,7 +93,11 @@ void fca_plan_opts_default(fca_plan_opts *opts /* HOST, out */);
  *
  * Runs GPU kernels on `stream`, then synchronises the stream once to read back
  * the sizes of the forest and work lists and allocates the plan's device
- * workspace (cudaMalloc).  The input buffers may be reused once it returns.
+ * workspace.  Plans allocate, in stream order on `stream`, from a memory pool
+ * the library creates per device on first use and never trims: memory that
+ * destroyed plans return stays in the pool (at most the largest total of
+ * plans alive at once) and makes the next plan's allocation free of page
+ * mapping.  The input buffers may be reused once it returns.
  * Errors: FCA_ERR_INVALID_ARG (shapes, a seq_len out of range),
  * FCA_ERR_BAD_BLOCK_ID (a referenced id out of range), FCA_ERR_UNSUPPORTED,
  * FCA_ERR_CUDA, FCA_ERR_OOM.  num_requests <= 16384, max_blocks <= 1 << 20.
@@ -189,7 +193,8 @@ fca_status fca_plan_export(fca_plan_t plan, int32_t *a, int32_t *b, int32_t *par
 /* Total member entries over all groups (HOST out). */
 fca_status fca_plan_member_count(fca_plan_t plan, int64_t *count);
 
-/* Free a plan and its device workspace (synchronises the device). NULL is ok. */
+/* Free a plan (synchronises the device first); its device workspace goes
+ * back to the library's plan pool.  NULL is ok. */
 fca_status fca_plan_destroy(fca_plan_t plan);
 
 /*

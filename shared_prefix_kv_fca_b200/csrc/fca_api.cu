@@ -80,8 +80,11 @@ void fca_plan_opts_default(fca_plan_opts* opts) {
 
 fca_status fca_plan_destroy(fca_plan_t plan) {
     if (!plan) return FCA_OK;
+    // the plan's memory goes back to the library's pool once nothing that may
+    // read it is still running
     cudaDeviceSynchronize();
-    for (void* p : plan->dev_allocs) cudaFree(p);
+    for (void* p : plan->dev_allocs) cudaFreeAsync(p, cudaStreamLegacy);
+    cudaStreamSynchronize(cudaStreamLegacy);
     if (plan->aux_stream) cudaStreamDestroy(plan->aux_stream);
     if (plan->ev_fork) cudaEventDestroy(plan->ev_fork);
     if (plan->ev_join) cudaEventDestroy(plan->ev_join);

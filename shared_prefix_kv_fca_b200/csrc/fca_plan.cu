@@ -33,6 +33,7 @@
 // Canonical order of the output: groups by (first block, smallest member);
 // members ascending.  One CTA sorts the groups in shared memory.
 #include <algorithm>
+#include <mutex>
 #include <cstdio>
 #include <cstring>
 #include <vector>
@@ -703,41 +704,78 @@ __global__ void k_fill_suffix_items(int32_t R, const int32_t* seq_lens, const in
 
 // ------------------------------------------------------------ host helpers
 
-// Stream-ordered temporaries, returned to the pool on scope exit.
-struct TempBuffers {
-    cudaStream_t stream;
-    std::vector<void*> ptrs;
-    bool ok = true;
-    explicit TempBuffers(cudaStream_t s) : stream(s) {}
-    ~TempBuffers() {
-        for (void* p : ptrs) cudaFreeAsync(p, stream);
-    }
-    template <typename T>
-    T* alloc(size_t count) {
-        void* p = nullptr;
-        if (cudaMallocAsync(&p, std::max<size_t>(count, 1) * sizeof(T), stream) != cudaSuccess) {
-            ok = false;
-            (void)cudaGetLastError();
-            return nullptr;
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// The memory pool plans allocate from, one per device, created on first use.
+// Its release threshold is unbounded: memory a destroyed plan gave back stays
+// mapped in the pool for the next plan instead of being unmapped at the next
+// synchronisation, so building a plan per decode step costs no page mapping.
+cudaError_t plan_pool(cudaMemPool_t* out) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mutex;
+    static cudaMemPool_t pools[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mutex);
+    if (!pools[dev]) {
+        cudaMemPoolProps props{};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        e = cudaMemPoolCreate(&pool, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = ~uint64_t(0);
+        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) {
+            cudaMemPoolDestroy(pool);
+            return e;
         }
-        ptrs.push_back(p);
-        return static_cast<T*>(p);
+        pools[dev] = pool;
+    }
+    *out = pools[dev];
+    return cudaSuccess;
+}
+
+// Lays arrays out back to back (256-byte aligned) in one allocation from the
+// library's plan pool: add() records where each array goes, commit() makes
+// the one stream-ordered allocation and sets the pointers.
+struct Arena {
+    struct Slot {
+        void** dst;
+        size_t off;
+    };
+    std::vector<Slot> slots;
+    size_t bytes = 0;
+    template <typename T>
+    size_t add(T** dst, size_t count) {
+        const size_t off = bytes;
+        slots.push_back({reinterpret_cast<void**>(dst), off});
+        bytes += align256(std::max<size_t>(count, 1) * sizeof(T));
+        return off;
+    }
+    cudaError_t commit(cudaStream_t stream, void** base) {
+        cudaMemPool_t pool = nullptr;
+        cudaError_t e = plan_pool(&pool);
+        if (e != cudaSuccess) return e;
+        e = cudaMallocFromPoolAsync(base, bytes, pool, stream);
+        if (e != cudaSuccess) return e;
+        for (const Slot& sl : slots) *sl.dst = static_cast<uint8_t*>(*base) + sl.off;
+        return cudaSuccess;
     }
 };
 
-template <typename T>
-T* plan_alloc(fca_plan_s* P, size_t count, bool& ok) {
-    void* p = nullptr;
-    const size_t bytes = std::max<size_t>(count, 1) * sizeof(T);
-    if (note_cuda(cudaMalloc(&p, bytes)) != cudaSuccess) {
-        ok = false;
-        (void)cudaGetLastError();
-        return nullptr;
+// Planner temporaries: one allocation, returned to the pool in stream order.
+struct TempArena {
+    cudaStream_t stream;
+    void* base = nullptr;
+    explicit TempArena(cudaStream_t s) : stream(s) {}
+    ~TempArena() {
+        if (base) cudaFreeAsync(base, stream);
     }
-    P->dev_allocs.push_back(p);
-    P->workspace_bytes += bytes;
-    return static_cast<T*>(p);
-}
+};
 
 int grid_for(int64_t work, int threads) {
     int64_t g = (work + threads - 1) / threads;
@@ -769,57 +807,72 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     const fca_plan_opts& opts = P->opts;
     const bool flat = P->flat;
 
-    TempBuffers tmp(stream);
+    // Temporaries.  The arrays that start at zero are laid out back to back
+    // (count .. hdr) so that one memset clears them.
     PlanScratch s{};
-    s.nfull = tmp.alloc<int32_t>(R);
-    s.owner = tmp.alloc<int32_t>(num_blocks);
-    s.count = tmp.alloc<int32_t>(num_blocks);
-    s.pos = tmp.alloc<int32_t>(num_blocks);
-    s.valid = tmp.alloc<int32_t>(num_blocks);
-    s.n_emit = tmp.alloc<int32_t>(R);
-    s.fill = tmp.alloc<int32_t>(R);
-    s.n_raw = tmp.alloc<int32_t>(1);
-    s.raw = tmp.alloc<RawGroup>(R);
-    s.keys = tmp.alloc<uint64_t>(R);
-    s.g_item_off = tmp.alloc<int32_t>(R + 1);
-    s.s_item_off = tmp.alloc<int32_t>(R + 1);
-    s.hdr = tmp.alloc<PlanHeader>(1);
-    bool ok = tmp.ok;
-    P->bt = plan_alloc<int32_t>(P, (size_t)R * max_blocks, ok);
-    P->seq_lens = plan_alloc<int32_t>(P, R, ok);
-    P->suffix_start = plan_alloc<int32_t>(P, R, ok);
-    P->g_a = plan_alloc<int32_t>(P, R, ok);
-    P->g_b = plan_alloc<int32_t>(P, R, ok);
-    P->g_parent = plan_alloc<int32_t>(P, R, ok);
-    P->g_nm = plan_alloc<int32_t>(P, R, ok);
-    P->g_moff = plan_alloc<int32_t>(P, R + 1, ok);
-    P->g_nch = plan_alloc<int32_t>(P, R, ok);
-    P->g_part = plan_alloc<int32_t>(P, R + 1, ok);
-    P->s_nch = plan_alloc<int32_t>(P, R, ok);
-    P->s_part = plan_alloc<int32_t>(P, R + 1, ok);
-    P->g_chunk = plan_alloc<int32_t>(P, R, ok);
-    P->s_chunk = plan_alloc<int32_t>(P, R, ok);
-    P->sched = plan_alloc<int32_t>(P, 4, ok);
-    int32_t* bin_cursor = tmp.alloc<int32_t>(kBins);
-    P->chain_off = plan_alloc<int32_t>(P, R + 1, ok);
-    P->dev_status = plan_alloc<int32_t>(P, 1, ok);
-    if (!ok) return FCA_ERR_OOM;
+    int32_t* bin_cursor = nullptr;
+    Arena ta;
+    ta.add(&s.owner, num_blocks);
+    ta.add(&s.pos, num_blocks);
+    const size_t zero0 = ta.add(&s.count, num_blocks);
+    ta.add(&s.valid, num_blocks);
+    ta.add(&s.n_emit, R);
+    ta.add(&s.fill, R);
+    ta.add(&s.n_raw, 1);
+    ta.add(&s.hdr, 1);
+    const size_t zero1 = ta.bytes;
+    ta.add(&s.nfull, R);
+    ta.add(&s.raw, R);
+    ta.add(&s.keys, R);
+    ta.add(&s.g_item_off, R + 1);
+    ta.add(&s.s_item_off, R + 1);
+    ta.add(&bin_cursor, kBins);
+    TempArena tmp(stream);
+    if (ta.commit(stream, &tmp.base) != cudaSuccess) {
+        tmp.base = nullptr;
+        (void)cudaGetLastError();
+        return FCA_ERR_OOM;
+    }
+
+    // The plan's arrays whose sizes are known before the planner runs
+    // (suffix_start, dev_status and sched start at zero and come first).
+    Arena pa;
+    pa.add(&P->suffix_start, R);
+    pa.add(&P->dev_status, 1);
+    pa.add(&P->sched, 4);
+    const size_t pzero = pa.bytes;
+    pa.add(&P->bt, (size_t)R * max_blocks);
+    pa.add(&P->seq_lens, R);
+    pa.add(&P->g_a, R);
+    pa.add(&P->g_b, R);
+    pa.add(&P->g_parent, R);
+    pa.add(&P->g_nm, R);
+    pa.add(&P->g_moff, R + 1);
+    pa.add(&P->g_nch, R);
+    pa.add(&P->g_part, R + 1);
+    pa.add(&P->s_nch, R);
+    pa.add(&P->s_part, R + 1);
+    pa.add(&P->g_chunk, R);
+    pa.add(&P->s_chunk, R);
+    pa.add(&P->chain_off, R + 1);
+    {
+        void* base = nullptr;
+        if (pa.commit(stream, &base) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return FCA_ERR_OOM;
+        }
+        P->dev_allocs.push_back(base);
+        P->workspace_bytes += pa.bytes;
+    }
     s.row_goff = P->chain_off;
 
     FCA_CK(cudaMemcpyAsync(P->bt, block_tables, sizeof(int32_t) * (size_t)R * max_blocks,
                            cudaMemcpyDeviceToDevice, stream));
     FCA_CK(cudaMemcpyAsync(P->seq_lens, seq_lens, sizeof(int32_t) * R, cudaMemcpyDeviceToDevice, stream));
     FCA_CK(cudaMemsetAsync(s.owner, 0x7F, sizeof(int32_t) * (size_t)num_blocks, stream));
-    FCA_CK(cudaMemsetAsync(s.count, 0, sizeof(int32_t) * (size_t)num_blocks, stream));
     FCA_CK(cudaMemsetAsync(s.pos, 0xFF, sizeof(int32_t) * (size_t)num_blocks, stream));
-    FCA_CK(cudaMemsetAsync(s.valid, 0, sizeof(int32_t) * (size_t)num_blocks, stream));
-    FCA_CK(cudaMemsetAsync(s.n_raw, 0, sizeof(int32_t), stream));
-    FCA_CK(cudaMemsetAsync(s.fill, 0, sizeof(int32_t) * R, stream));
-    FCA_CK(cudaMemsetAsync(s.n_emit, 0, sizeof(int32_t) * R, stream));
-    FCA_CK(cudaMemsetAsync(s.hdr, 0, sizeof(PlanHeader), stream));
-    FCA_CK(cudaMemsetAsync(P->suffix_start, 0, sizeof(int32_t) * R, stream));
-    FCA_CK(cudaMemsetAsync(P->dev_status, 0, sizeof(int32_t), stream));
-    FCA_CK(cudaMemsetAsync(P->sched, 0, 4 * sizeof(int32_t), stream));
+    FCA_CK(cudaMemsetAsync(static_cast<uint8_t*>(tmp.base) + zero0, 0, zero1 - zero0, stream));
+    FCA_CK(cudaMemsetAsync(P->suffix_start, 0, pzero, stream));
 
     const int64_t cells = (int64_t)R * max_blocks;
     k_validate<<<grid_for(cells, 256), 256, 0, stream>>>(P->bt, max_blocks, P->seq_lens, R, num_blocks, s.nfull,
@@ -897,14 +950,24 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     const int64_t n_part = (int64_t)H.n_prefix_partials + H.n_suffix_partials;
     if (n_part >= (int64_t)INT32_MAX / 2) return FCA_ERR_UNSUPPORTED;
 
-    P->members = plan_alloc<int32_t>(P, H.n_member_entries, ok);
-    P->chain_g = plan_alloc<int32_t>(P, H.n_chain_entries, ok);
-    P->chain_pos = plan_alloc<int32_t>(P, H.n_chain_entries, ok);
-    P->prefix_items = plan_alloc<PrefixItem>(P, H.n_prefix_items, ok);
-    P->suffix_items = plan_alloc<SuffixItem>(P, H.n_suffix_items, ok);
-    P->part_o = plan_alloc<float>(P, (size_t)n_part * D, ok);
-    P->part_lse = plan_alloc<float>(P, n_part, ok);
-    if (!ok) return FCA_ERR_OOM;
+    // the arrays sized by the planner
+    Arena wa;
+    wa.add(&P->members, H.n_member_entries);
+    wa.add(&P->chain_g, H.n_chain_entries);
+    wa.add(&P->chain_pos, H.n_chain_entries);
+    wa.add(&P->prefix_items, H.n_prefix_items);
+    wa.add(&P->suffix_items, H.n_suffix_items);
+    wa.add(&P->part_lse, n_part);
+    wa.add(&P->part_o, (size_t)n_part * D);
+    {
+        void* base = nullptr;
+        if (wa.commit(stream, &base) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return FCA_ERR_OOM;
+        }
+        P->dev_allocs.push_back(base);
+        P->workspace_bytes += wa.bytes;
+    }
 
     if (!flat && H.n_groups > 0) {
         ra.pass = 1;
