@@ -145,6 +145,43 @@ def gpu_id_for(local_rank: int) -> str:
     return str(local_rank)
 
 
+# ------------------------------------------------------------------ ranks
+
+class RankReducer:
+    """Max / sum of one float over all ranks; the identity at world size 1.
+    Every rank must make the same calls in the same order."""
+
+    def __init__(self, world: int, device=None):
+        self.world = world
+        self.device = device
+
+    def _reduce(self, x: float, op) -> float:
+        if self.world == 1:
+            return float(x)
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=op)
+        return float(t.item())
+
+    def max(self, x: float) -> float:
+        import torch.distributed as dist
+        return self._reduce(x, dist.ReduceOp.MAX)
+
+    def sum(self, x: float) -> float:
+        import torch.distributed as dist
+        return self._reduce(x, dist.ReduceOp.SUM)
+
+
+def aggregate_step(step_ms: float, unique_bytes_rank: int, red: RankReducer):
+    """Whole-job throughput of one step: the unique KV bytes every rank
+    processed over the slowest rank's step time.  Returns (max step ms,
+    total bytes, GB/s)."""
+    step = red.max(step_ms)
+    total = red.sum(unique_bytes_rank)
+    return step, total, total / (step * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ oracle legs
 
 def oracle_sample(w, budget_s: float, seed: int = 0):
@@ -258,19 +295,8 @@ def fca_arm(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def sum_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+    red = RankReducer(world, dev)
+    max_over_ranks, sum_over_ranks = red.max, red.sum
 
     w = fca_workloads.make(args.config, seed=rank, prompts=args.prompts)
     q, k, v, bt, sl = w.torch_inputs(dev)
@@ -336,12 +362,12 @@ def fca_arm(args):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    step_ms = run_steps(plan, args.steps, True)
+    step_ms_rank = run_steps(plan, args.steps, True)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop() if sampler else None
     barrier()
     assert fca.fca_check_device_status(plan, stream) == 0
-    step_ms = max_over_ranks(step_ms)
+    step_ms, total_unique, value = aggregate_step(step_ms_rank, st["unique_kv_bytes"], red)
     n_launch = (1 if (st["prefix_items"] > 0) else 0) + (1 if st["suffix_items"] > 0 else 0) + 1
 
     # ---- the passes one at a time (per-kernel roofline)
@@ -402,9 +428,7 @@ def fca_arm(args):
                "includes": "H2D of q and block tables, fca_plan (one host sync), fca_decode, "
                            "D2H of out and lse; the KV cache is resident state"}
 
-    total_unique = sum_over_ranks(st["unique_kv_bytes"])
     peak, peak_kind = peaks()
-    value = total_unique / (step_ms * 1e-3) / 1e9
 
     # dominant kernel and its roofline
     pass_ms = {key: max_over_ranks(fca_t[key]) for key in ("prefix", "suffix", "merge")}

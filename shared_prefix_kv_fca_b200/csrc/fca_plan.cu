@@ -649,7 +649,7 @@ __global__ void __launch_bounds__(256) k_sort_members(const PlanHeader* hdr, con
 
 // ------------------------------------------------------------ work lists
 
-// One CTA per group: items (head, q-tile, chunk), heads outermost.
+// One CTA per group: items (q-tile, chunk, head), heads innermost.
 __global__ void k_fill_prefix_items(const PlanHeader* hdr, const int32_t* g_a, const int32_t* g_b,
                                     const int32_t* g_nm, const int32_t* g_moff, const int32_t* g_nch,
                                     const int32_t* g_chunk, const int32_t* g_part, const int32_t* item_off,
