@@ -535,10 +535,13 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
     const int64_t n_members = block_exclusive_scan(n, [&](int32_t i) { return (int64_t)A.g_nm[i]; },
                                                    A.g_moff, red);
     for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+        // chunks are whole stages of the grouped pass; their count follows
+        // from the rounded size, so that every chunk holds tokens
         const int32_t tok = (A.g_b[i] - A.g_a[i]) * kBlockSize;
-        const int32_t nch = (tok + split_p - 1) / split_p;
-        A.g_nch[i] = nch;
-        A.g_chunk[i] = ((tok + nch - 1) / nch + kStageTokens - 1) / kStageTokens * kStageTokens;
+        const int32_t want = (tok + split_p - 1) / split_p;
+        const int32_t chunk = ((tok + want - 1) / want + kStageTokens - 1) / kStageTokens * kStageTokens;
+        A.g_chunk[i] = chunk;
+        A.g_nch[i] = (tok + chunk - 1) / chunk;
     }
     __syncthreads();
     const int64_t n_pitems = block_exclusive_scan(

@@ -34,6 +34,8 @@
 //               the first stages is rare (numerator and denominator use the
 //               same reference, so the result is exact).  At the end of an
 //               item the two partial states are merged by their weights.
+// Warps whose 32 tile rows are all past the group's stacked rows skip the
+// softmax and the output, and keep only the barrier protocol.
 // Output: one partial row (normalised o, natural-log lse) per stacked query
 // row, merged later with the row's other partials.
 #include <algorithm>
@@ -342,12 +344,28 @@ __global__ void __launch_bounds__(kPreThreads, 1)
             const bool has_next = item + item_step < a.n_items;
             float m_ref = -INFINITY, l_run = 0.f;
             int32_t my_last = -1;                      // my last stage of this item (global index)
+            // A warp whose 32 tile rows are all past the group's stacked rows has
+            // nothing to compute: it skips the softmax and the output, and keeps
+            // only the barrier protocol (its P and O rows are never read back).
+            const bool live = quarter * 32 < it.nrows;
             for (int32_t j = ((g & 1) == (uint32_t)wg) ? 0 : 1; j < ns; j += 2) {
                 const uint32_t gg = g + j;
                 my_last = (int32_t)gg;
                 bool got = dev::mbar_wait(&s_full[wg], (gg >> 1) & 1, abort_flag, a.err);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 dev::tc_fence_after();
+                if (!live) {
+                    // same arrivals in the same order as a live warp; p_free first,
+                    // so that this arrival cannot count towards an earlier phase
+                    dev::mbar_arrive(&s_free[wg]);
+                    if (gg >= 2) {
+                        got = dev::mbar_wait(&p_free[wg], ((gg >> 1) - 1) & 1, abort_flag, a.err);
+                        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                    }
+                    dev::mbar_arrive(&p_full[wg]);
+                    if (j + 1 == ns && has_next) load_q(a.items[item + item_step]);
+                    continue;
+                }
                 const int32_t n_valid = min(kStageTokens, n_tok - j * kStageTokens);
                 float x[64];
 #pragma unroll
@@ -447,7 +465,7 @@ __global__ void __launch_bounds__(kPreThreads, 1)
             const bool row_valid = r < it.nrows;
             float* dst = a.part_o + ((int64_t)it.part_row0 + r) * D + wg * kOHalf;
 #pragma unroll
-            for (int c = 0; c < kOHalf / 16; ++c) {
+            for (int c = 0; live && c < kOHalf / 16; ++c) {
                 uint32_t o0[16], o1[16];
                 dev::tmem_ld16(tmem + lane_base + L::kColO + wg * kOHalf + c * 16, o0);
                 dev::tmem_ld16(tmem + lane_base + L::kColO + D + wg * kOHalf + c * 16, o1);

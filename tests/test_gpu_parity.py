@@ -199,7 +199,7 @@ def test_prefix_rescale_path(split):
 def test_many_items_per_cta():
     # far more grouped-pass items than SMs: every CTA walks several items
     for seed in (1, 2):
-        w = fca_workloads.make("llama8b", seed=seed, prompts=4)
+        w = fca_workloads.make("llama8b", seed=seed, prompts=8)
         o, l, _, st = run(w, split_tokens=64)
         assert st["prefix_items"] > 4 * 148
         pairs = sampled_pairs(w, 64, seed)
