@@ -72,6 +72,7 @@ struct PlanHeader {
     int64_t flat_kv_tokens;
     int64_t prefix_tok_sum;     // sum over groups of their token count
     int64_t suffix_tok_sum;
+    int64_t prefix_tile_tok_sum;// sum over groups of token count x 128-row query tiles
 };
 
 // Remember e (if it is an error) as the calling thread's last CUDA error.

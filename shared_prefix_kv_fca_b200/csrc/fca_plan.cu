@@ -519,7 +519,9 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
     }
     for (int32_t r = threadIdx.x; r < R; r += blockDim.x)
         ws += A.seq_lens[r] - (int64_t)A.suffix_start[r] * kBlockSize;
-    wp = block_sum64(wp, red) * A.Hkv;
+    wp = block_sum64(wp, red);
+    if (threadIdx.x == 0) hdr->prefix_tile_tok_sum = wp;
+    wp *= A.Hkv;
     ws = block_sum64(ws, red) * A.Hkv;
     int32_t split_p = A.split_opt, split_s = A.split_opt;
     if (split_p <= 0) {
