@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-flat", action="store_true")
+    ap.add_argument("--layers", type=int, default=1,
+                    help="also time a multi-layer step: one plan, then this many layers' decodes")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0,
                     help="approximate CPU seconds of the oracle baseline sample")
     return ap.parse_args()
@@ -428,6 +430,40 @@ def fca_arm(args):
                "includes": "H2D of q and block tables, fca_plan (one host sync), fca_decode, "
                            "D2H of out and lse; the KV cache is resident state"}
 
+    # ---- a model-shaped step: one plan serves every layer
+    multi = None
+    if args.layers > 1:
+        ks = [k] + [k.clone() for _ in range(args.layers - 1)]
+        vs = [v] + [v.clone() for _ in range(args.layers - 1)]
+
+        def layers_step():
+            p = fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, split_tokens=args.split, stream=stream)
+            for kl, vl in zip(ks, vs):
+                fca.fca_decode(q, kl, vl, p, out, lse, w.scale, stream)
+            return p
+
+        for _ in range(max(1, args.warmup)):
+            flush.zero_()
+            layers_step().close()
+        barrier()
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            p = layers_step()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+            p.close()
+        ml_ms = max_over_ranks(statistics.mean(times))
+        del ks, vs
+        multi = {"layers": args.layers, "ms_per_step": ml_ms,
+                 "unique_kv_gbs": args.layers * sum_over_ranks(st["unique_kv_bytes"]) / (ml_ms * 1e-3) / 1e9,
+                 "plan_and_launch_share": max(0.0, 1.0 - args.layers * step_ms / ml_ms),
+                 "includes": "fca_plan (one host sync) then one fca_decode per layer over distinct caches"}
+
     peak, peak_kind = peaks()
 
     # dominant kernel and its roofline
@@ -468,7 +504,7 @@ def fca_arm(args):
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_bytes": alg_bytes[dominant],
                          "peak_note": f"{peak_kind} copy bandwidth (MEASURED_PEAKS hbm_gbs)"},
-            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "multilayer": multi,
             "gpu_launches": n_launch * args.steps, "impl": "fca",
         }
         print(json.dumps(line), flush=True)

@@ -154,6 +154,31 @@ def test_tiny_config_all_outputs():
         assert_close(o, l, o_ref, l_ref, f"tiny flat={flat}")
 
 
+def test_one_plan_serves_several_layers():
+    # the plan depends only on the block tables and lengths: every layer of a
+    # model reuses it with that layer's q and caches
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    w = fca_workloads.random_small(5, Hq=8, Hkv=2, D=128, max_requests=16)
+    bt = torch.from_numpy(w.block_tables).cuda()
+    sl = torch.from_numpy(w.seq_lens).cuda()
+    with fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D) as plan:
+        for layer in range(3):
+            q = fca_workloads.normal_bf16(w.q.shape, 200 + layer, 0)
+            k = fca_workloads.normal_bf16(w.k_cache.shape, 200 + layer, 1)
+            v = fca_workloads.normal_bf16(w.v_cache.shape, 200 + layer, 2)
+            lw = fca_workloads.Workload(f"layer{layer}", q, k, v, w.block_tables, w.seq_lens, w.Hq, w.Hkv,
+                                        w.D, w.block_size, 200 + layer)
+            qd, kd, vd, _, _ = lw.torch_inputs("cuda")
+            out = torch.empty_like(qd)
+            lse = torch.empty(w.R, w.Hq, dtype=torch.float32, device="cuda")
+            fca.fca_decode(qd, kd, vd, plan, out, lse, w.scale)
+            assert fca.fca_check_device_status(plan) == 0
+            o_ref, l_ref = oracle.paged_attention(q, k, v, w.block_tables, w.seq_lens, w.scale)
+            assert_close(out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
+                         o_ref, l_ref, f"layer {layer}")
+
+
 def test_lse_optional():
     w = fca_workloads.random_small(4, D=64)
     o, l, _, _ = run(w, lse=False)
