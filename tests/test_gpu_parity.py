@@ -135,6 +135,31 @@ def test_decode_matches_oracle_random(seed, flat):
     assert_close(o, l, o_ref, l_ref, f"seed {seed} flat={flat}")
 
 
+@pytest.mark.parametrize("shape", [(16, 1, 128), (32, 2, 64), (16, 1, 64), (12, 1, 128)])
+@pytest.mark.parametrize("flat", [False, True])
+def test_decode_wide_gqa(shape, flat):
+    # 9 to 16 query heads per KV head: the per-request pass's second column
+    # tile, and group tiles of 16 rows per member
+    Hq, Hkv, D = shape
+    for seed in (21, 22, 23):
+        w = fca_workloads.random_small(seed, Hq=Hq, Hkv=Hkv, D=D, max_requests=20, poison_padding=True)
+        o, l, _, _ = run(w, flat=flat)
+        o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+        assert_close(o, l, o_ref, l_ref, f"gqa {shape} seed {seed} flat={flat}")
+
+
+def test_decode_one_group_of_many_members():
+    # one prompt shared by 40 requests x 16 query heads = 640 stacked rows:
+    # five 128-row tiles of one group
+    rng = np.random.default_rng(9)
+    reqs = [[("p", 300), (None, int(rng.integers(1, 40)))] for _ in range(40)]
+    w = fca_workloads.fill("wide", reqs, Hq=16, Hkv=1, D=128, seed=9, rng=rng, poison_padding=True)
+    o, l, exp, st = run(w)
+    assert len(exp["a"]) == 1 and st["prefix_items"] >= 5
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(o, l, o_ref, l_ref, "one wide group")
+
+
 @pytest.mark.parametrize("split", [64, 128, 256])
 def test_decode_small_splits(split):
     # many split chunks per group and per request, ragged tails

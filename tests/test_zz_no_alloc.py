@@ -114,6 +114,12 @@ def test_static_matches_flat_decode_small(seed):
 
 
 @pytest.mark.gpu
+def test_static_matches_flat_decode_wide_gqa():
+    w = fca_workloads.random_small(31, Hq=16, Hkv=1, D=128, max_requests=16, poison_padding=True)
+    _two_calls_match_flat(w, check_oracle=True)
+
+
+@pytest.mark.gpu
 def test_static_matches_flat_decode_head_dim_64():
     _two_calls_match_flat(fca_workloads.make("tiny"), check_oracle=True)
 
