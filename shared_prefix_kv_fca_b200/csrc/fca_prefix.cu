@@ -11,29 +11,39 @@
 // Work item = (group, KV head, 128-row Q tile, token chunk).  The kernel is
 // persistent: one CTA per SM walks its items (blockIdx.x, +gridDim.x, ...),
 // tensor memory is allocated once, and the K/V stream runs on across items.
-// 320 threads in three roles:
+// 352 threads in four roles:
 //   warp 0      TMA producer: 64-token stages of K and V (four paged 16-token
 //               blocks, 64-column halves, 128-byte swizzle) into a ring of
 //               kPreStages slots; blocks past a chunk are loaded from rows
 //               beyond the cache, which TMA fills with zeros;
-//   warp 1      allocates tensor memory and, from one thread, issues
-//               S = Q K^T (M=128, N=64) and O_w += P V (M=128, N=head_dim),
-//               signalling completions with tcgen05.commit.  Q and P are the
-//               A operands and live in tensor memory next to S and O, so all
-//               of shared memory holds the K/V ring (the stages a slow HBM
-//               stream needs in flight); a K slot is released as soon as its
-//               Q K^T has run, a V slot after its P V;
 //   warps 2-9   two softmax warpgroups, one thread per query row each.  Stage
 //               s of an item belongs to warpgroup s % 2, which has its own S
-//               buffer, P buffer, O accumulator and online-softmax state, so
-//               the two groups work on consecutive stages at the same time
-//               and never wait for each other inside an item.  fp32 max in
-//               the log2 domain; P stored to tensor memory as packed bf16.  A group's O accumulator is rescaled in
-//               tensor memory only when a row's maximum grows by more than
-//               2^kRescaleLog2 over the one its exponentials use, which after
-//               the first stages is rare (numerator and denominator use the
-//               same reference, so the result is exact).  At the end of an
-//               item the two partial states are merged by their weights.
+//               buffer, P buffer, O accumulator, copy of the Q tile and
+//               online-softmax state, so the two groups work on consecutive
+//               stages at the same time.  fp32 max in the log2 domain; P
+//               stored as packed bf16 in shared memory, in the 128-byte
+//               swizzled layout the MMA reads.  A group's O accumulator is
+//               rescaled in tensor memory only when a row's maximum grows by
+//               more than 2^kRescaleLog2 over the one its exponentials use,
+//               which after the first stages is rare (numerator and
+//               denominator use the same reference, so the result is exact).
+//               At the end of an item the two partial states are merged by
+//               their weights.  A group reloads its Q copy for its next item
+//               once it has read its own last S of the current one;
+//   warps 1, 10 one MMA issuer per softmax group (warp 1 also allocates
+//               tensor memory): S = Q K^T (M=128, N=64, Q from tensor memory)
+//               and O_w += P V (M=128, N=head_dim, P from shared memory, the
+//               faster form), completions signalled with tcgen05.commit.
+//               Issuing a tcgen05.mma returns about when the tensor core
+//               takes it, so a single issuer spends its barrier checks with
+//               the tensor core idle; two issuers overlap them.  Each issues
+//               its group's Q K^T of stage s + 2 as soon as the group has read
+//               S(s), before P V(s).
+// Barrier phases are waited by parity, so each waiter keeps within one phase
+// of its barrier: "full"/"empty" pairs are per group except the K/V ring,
+// whose slots the two issuers use alternately (an issuer first waits for a
+// slot's previous stage to be released), and "O read" is signalled per group
+// only for items in which the group has stages.
 // Warps whose 32 tile rows are all past the group's stacked rows skip the
 // softmax and the output, and keep only the barrier protocol.
 // Output: one partial row (normalised o, natural-log lse) per stacked query
@@ -49,9 +59,10 @@ namespace fca {
 
 namespace {
 
-constexpr int kPreStages = 6;
+constexpr int kPreStages = 5;
 constexpr int kSoftWarps = 8;
-constexpr int kPreThreads = 64 + kSoftWarps * 32;
+constexpr int kPreThreads = 96 + kSoftWarps * 32;     // producer, MMA issuer 0, 8 softmax warps, MMA issuer 1
+constexpr int kMmaWarp1 = 2 + kSoftWarps;             // the second MMA-issuing warp
 constexpr float kRescaleLog2 = 8.f;
 
 struct PrefixArgs {
@@ -74,19 +85,20 @@ struct PreLayout {
     static constexpr int kKV = kHalves * 64 * 128;        // one 64-token K (or V) stage
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kPreStages * kKV;
-    static constexpr int kOffX = kOffV + kPreStages * kKV; // per-row (m, l) of each group [2 items][2][2][128] f32
+    static constexpr int kOffP = kOffV + kPreStages * kKV; // P of group w: 128 rows x 64 tokens bf16 at + 16 KB w
+    static constexpr int kOffX = kOffP + 2 * 128 * 128;    // per-row (m, l) of each group [2 items][2][2][128] f32
     static constexpr int kOffBar = kOffX + 2 * 2 * 2 * 128 * 4;
-    // q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], s_free[2],
-    // p_full[2], p_free[2], o_full[2], o_free, mma_done, l_bar
-    static constexpr int kNumBars = 1 + 4 * kPreStages + 10 + 3;
+    // q_full[2], k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], s_free[2],
+    // p_full[2], p_free[2], o_full[2], o_free[2], mma_done[2], l_bar
+    static constexpr int kNumBars = 2 + 4 * kPreStages + 10 + 5;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kTotal = kOffMisc + 64 + 1024;   // + alignment slack
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0;                  // S of group w: 64 fp32 columns at 64 w
     static constexpr uint32_t kColO = 128;                // O of group w: D fp32 columns at 128 + D w
-    static constexpr uint32_t kColP = 128 + 2 * D;        // P of group w: 32 columns (64 bf16) at + 32 w
-    static constexpr uint32_t kColQ = kColP + 64;         // Q: D / 2 columns (D bf16)
-    static_assert(kColQ + D / 2 <= kTmemCols, "tensor memory budget");
+    static constexpr uint32_t kColQ = 128 + 2 * D;        // Q copy of group w: D / 2 columns at + (D / 2) w
+    static_assert(kColQ + D <= kTmemCols, "tensor memory budget");
+    static_assert(kTotal <= 227 * 1024, "shared memory budget");
 };
 
 __device__ __forceinline__ int32_t stages_of(const PrefixItem& it) {
@@ -100,8 +112,8 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
-    uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;
+    uint64_t* q_full = bars;             // [2]: Q copy of group w loaded
+    uint64_t* k_full = bars + 2;
     uint64_t* v_full = k_full + kPreStages;
     uint64_t* k_empty = v_full + kPreStages;
     uint64_t* v_empty = k_empty + kPreStages;
@@ -110,9 +122,9 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     uint64_t* p_full = s_free + 2;
     uint64_t* p_free = p_full + 2;
     uint64_t* o_full = p_free + 2;
-    uint64_t* o_free = o_full + 2;
-    uint64_t* mma_done = o_free + 1;
-    uint64_t* l_bar = mma_done + 1;      // end-of-item exchange of (m, l) between the groups
+    uint64_t* o_free = o_full + 2;       // [2]: the epilogue has read O of group w
+    uint64_t* mma_done = o_free + 2;     // [2]
+    uint64_t* l_bar = mma_done + 2;      // end-of-item exchange of (m, l) between the groups
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 16);
     float* xml = reinterpret_cast<float*>(smem + L::kOffX);
@@ -121,7 +133,8 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     const int32_t first_item = blockIdx.x, item_step = gridDim.x;
 
     if (threadIdx.x == 0) {
-        dev::mbar_init(q_full, 128);
+        dev::mbar_init(&q_full[0], 128);
+        dev::mbar_init(&q_full[1], 128);
         for (int st = 0; st < kPreStages; ++st) {
             dev::mbar_init(&k_full[st], 1);
             dev::mbar_init(&v_full[st], 1);
@@ -135,8 +148,10 @@ __global__ void __launch_bounds__(kPreThreads, 1)
             dev::mbar_init(&p_free[b], 1);
             dev::mbar_init(&o_full[b], 1);
         }
-        dev::mbar_init(o_free, kSoftWarps * 32);
-        dev::mbar_init(mma_done, 1);
+        dev::mbar_init(&o_free[0], kSoftWarps * 32);
+        dev::mbar_init(&o_free[1], kSoftWarps * 32);
+        dev::mbar_init(&mma_done[0], 1);
+        dev::mbar_init(&mma_done[1], 1);
         dev::mbar_init(l_bar, kSoftWarps * 32);
         *abort_flag = 0;
         dev::fence_mbarrier_init();
@@ -229,72 +244,93 @@ __global__ void __launch_bounds__(kPreThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == kMmaWarp1) {
+        // ------------------------------------------------ MMA issuers
+        // One thread per softmax group w issues that group's MMAs (its stages
+        // are those of parity w), so that one issuer's barrier checks overlap
+        // the other's MMAs.  Each thread's MMAs run in its issue order, and
+        // each commit covers only that thread's MMAs.
+        const int w = warp == 1 ? 0 : 1;
         if (lane == 0) {
             constexpr uint32_t idesc_qk = dev::idesc_bf16_f32(128, 64, false, false);
             constexpr uint32_t idesc_pv = dev::idesc_bf16_f32(128, D, false, true);
+            const uint32_t q_col = L::kColQ + w * (D / 2);
+            const uint32_t p_base = dev::smem_u32(smem + L::kOffP + w * 128 * 128);
+            // The K/V ring is shared by the two issuers, which take alternate
+            // stages: before a parity wait on a slot's "full" barrier, wait for
+            // the slot's previous stage (the other issuer's) to be released, so
+            // that the barrier cannot still be a phase behind and the parity
+            // wait cannot match the previous phase.
             auto issue_qk = [&](uint32_t gg) -> bool {
-                const int s = gg % kPreStages, sb = gg & 1;
+                const int s = gg % kPreStages;
+                if (gg >= kPreStages &&
+                    !dev::mbar_wait(&k_empty[s], ((gg / kPreStages) - 1) & 1, abort_flag, a.err))
+                    return false;
                 if (!dev::mbar_wait(&k_full[s], (gg / kPreStages) & 1, abort_flag, a.err)) return false;
-                if (gg >= 2 && !dev::mbar_wait(&s_free[sb], ((gg >> 1) - 1) & 1, abort_flag, a.err)) return false;
+                if (gg >= 2 && !dev::mbar_wait(&s_free[w], ((gg >> 1) - 1) & 1, abort_flag, a.err)) return false;
                 dev::tc_fence_after();
                 const uint32_t k_base = dev::smem_u32(smem + L::kOffK + s * L::kKV);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint64_t bd =
                         dev::smem_desc_sw128(k_base + (k >> 2) * (64 * 128) + (k & 3) * 32, 16, 1024);
-                    dev::tc_mma_ts(tmem + L::kColS + sb * 64, tmem + L::kColQ + k * 8, bd, idesc_qk, k > 0 ? 1u : 0u);
+                    dev::tc_mma_ts(tmem + L::kColS + w * 64, tmem + q_col + k * 8, bd, idesc_qk, k > 0 ? 1u : 0u);
                 }
-                dev::tc_commit(&s_full[sb]);
+                dev::tc_commit(&s_full[w]);
                 dev::tc_commit(&k_empty[s]);
                 return true;
             };
-            // first: the first P V of group (gg & 1) in this item, which starts
-            // its O accumulator afresh once the previous item's epilogue read it
-            auto issue_pv = [&](uint32_t gg, bool first, int32_t local_item) -> bool {
-                const int s = gg % kPreStages, pb = gg & 1;
-                if (!dev::mbar_wait(&p_full[pb], (gg >> 1) & 1, abort_flag, a.err)) return false;
-                if (first && local_item > 0 && !dev::mbar_wait(o_free, (local_item - 1) & 1, abort_flag, a.err))
+            // first: the group's first P V in the item, which starts its O
+            // accumulator afresh; q_item: how many earlier items had stages of
+            // this group.  o_free[w] completes once per such item, when its
+            // epilogue has read O of this group, so waiting on exactly the
+            // previous one keeps this thread and the barrier within one phase.
+            auto issue_pv = [&](uint32_t gg, bool first, int32_t q_item) -> bool {
+                const int s = gg % kPreStages;
+                if (!dev::mbar_wait(&p_full[w], (gg >> 1) & 1, abort_flag, a.err)) return false;
+                if (first && q_item > 0 && !dev::mbar_wait(&o_free[w], (q_item - 1) & 1, abort_flag, a.err))
+                    return false;
+                if (gg >= kPreStages &&
+                    !dev::mbar_wait(&v_empty[s], ((gg / kPreStages) - 1) & 1, abort_flag, a.err))
                     return false;
                 if (!dev::mbar_wait(&v_full[s], (gg / kPreStages) & 1, abort_flag, a.err)) return false;
                 dev::tc_fence_after();
                 const uint32_t v_base = dev::smem_u32(smem + L::kOffV + s * L::kKV);
 #pragma unroll
                 for (int k = 0; k < kStageTokens / 16; ++k) {
+                    const uint64_t ad = dev::smem_desc_sw128(p_base + k * 32, 16, 1024);
                     const uint64_t bd = dev::smem_desc_sw128(v_base + k * 2048, 64 * 128, 1024);
-                    dev::tc_mma_ts(tmem + L::kColO + pb * D, tmem + L::kColP + pb * 32 + k * 8, bd, idesc_pv,
-                                   (first && k == 0) ? 0u : 1u);
+                    dev::tc_mma_ss(tmem + L::kColO + w * D, ad, bd, idesc_pv, (first && k == 0) ? 0u : 1u);
                 }
-                dev::tc_commit(&o_full[pb]);
-                dev::tc_commit(&p_free[pb]);
+                dev::tc_commit(&o_full[w]);
+                dev::tc_commit(&p_free[w]);
                 dev::tc_commit(&v_empty[s]);
                 return true;
             };
             bool ok = true;
             uint32_t g = 0;
-            int32_t local = 0;
-            if (first_item < a.n_items) ok = dev::mbar_wait(q_full, 0, abort_flag, a.err) && issue_qk(0);
+            int32_t local = 0, q_items = 0;
             for (int32_t item = first_item; ok && item < a.n_items; item += item_step, ++local) {
                 const int32_t ns = stages_of(a.items[item]);
-                const bool has_next = item + item_step < a.n_items;
-                for (int32_t j = 0; ok && j < ns; ++j) {
-                    const uint32_t gg = g + j;
-                    if (j + 1 < ns) {
-                        ok = issue_qk(gg + 1) && issue_pv(gg, j < 2, local);
-                    } else {
-                        // last stage: finish this item's O first, then start the next item
-                        ok = issue_pv(gg, j < 2, local);
-                        if (ok && has_next)
-                            ok = dev::mbar_wait(q_full, (local + 1) & 1, abort_flag, a.err) && issue_qk(gg + 1);
+                const int32_t j0 = ((g & 1) == (uint32_t)w) ? 0 : 1;
+                if (j0 < ns) {
+                    // this group's Q copy holds the item's queries once q_full[w] completes
+                    const int32_t q_item = q_items++;
+                    ok = dev::mbar_wait(&q_full[w], q_item & 1, abort_flag, a.err) && issue_qk(g + j0);
+                    for (int32_t j = j0; ok && j < ns; j += 2) {
+                        const uint32_t gg = g + j;
+                        // S(gg + 2) reuses the buffer of S(gg), which the group reads
+                        // first thing in stage gg: that Q K^T runs during its softmax
+                        if (j + 2 < ns) ok = issue_qk(gg + 2);
+                        ok = ok && issue_pv(gg, j < 2, q_item);
                     }
                 }
                 g += ns;
             }
             // every MMA of this thread has retired before tensor memory is freed
-            dev::tc_commit(mma_done);
+            dev::tc_commit(&mma_done[w]);
             volatile int never = 0;
-            dev::mbar_wait(mma_done, 0, &never, a.err);
+            dev::mbar_wait(&mma_done[w], 0, &never, a.err);
         }
         __syncwarp();
     } else {
@@ -327,21 +363,32 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                     w[e * 4 + 2] = v.z;
                     w[e * 4 + 3] = v.w;
                 }
-                dev::tmem_st32(tmem + lane_base + L::kColQ + c * 32, w);
+                dev::tmem_st32(tmem + lane_base + L::kColQ + wg * (D / 2) + c * 32, w);
             }
             dev::tc_wait_st();
             dev::tc_fence_before();
-            dev::mbar_arrive(q_full);
+            dev::mbar_arrive(&q_full[wg]);
         };
+        // this group has stages in an item of ns stages that starts at global stage gs
+        auto has_stages = [&](int32_t ns, uint32_t gs) { return (((gs & 1) == (uint32_t)wg) ? 0 : 1) < ns; };
 
         bool ok = true;
         uint32_t g = 0;
         int32_t local = 0;
-        if (wg == 0 && first_item < a.n_items) load_q(a.items[first_item]);
+        int32_t q_item = -1;                           // item whose queries this group's Q copy holds
         for (int32_t item = first_item; ok && item < a.n_items; item += item_step, ++local) {
             const PrefixItem it = a.items[item];
             const int32_t ns = stages_of(it), n_tok = it.tok1 - it.tok0;
-            const bool has_next = item + item_step < a.n_items;
+            const int32_t next = item + item_step;
+            // Q of the next item, if this group has stages there: loaded after the
+            // group's last S of this item, when all of its Q K^T have completed
+            const bool load_next = next < a.n_items && has_stages(stages_of(a.items[next]), g + ns);
+            // groups with stages in this item (their issuers wait for this epilogue)
+            const bool had0 = (((g & 1) == 0u) ? 0 : 1) < ns, had1 = (((g & 1) == 1u) ? 0 : 1) < ns;
+            if (has_stages(ns, g) && q_item != item) {
+                load_q(it);
+                q_item = item;
+            }
             float m_ref = -INFINITY, l_run = 0.f;
             int32_t my_last = -1;                      // my last stage of this item (global index)
             // A warp whose 32 tile rows are all past the group's stacked rows has
@@ -363,7 +410,10 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                     }
                     dev::mbar_arrive(&p_full[wg]);
-                    if (j + 1 == ns && has_next) load_q(a.items[item + item_step]);
+                    if (j + 2 >= ns && load_next) {
+                        load_q(a.items[next]);
+                        q_item = next;
+                    }
                     continue;
                 }
                 const int32_t n_valid = min(kStageTokens, n_tok - j * kStageTokens);
@@ -429,13 +479,18 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                     pw[i] = dev::pack_bf16x2(p0, p1);
                 }
                 l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                dev::tmem_st32(tmem + lane_base + L::kColP + wg * 32, pw);
-                dev::tc_wait_st();
-                dev::tc_fence_before();
+                // row r of P, 64 tokens = eight 16-byte chunks, 128-byte swizzle
+                uint8_t* prow = smem + L::kOffP + wg * 128 * 128 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+                        make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+                dev::fence_proxy_async_smem();
                 dev::mbar_arrive(&p_full[wg]);
-                // the group that read the item's last S knows every Q K^T of the
-                // item has completed: it refills the Q tile for the next item
-                if (j + 1 == ns && has_next) load_q(a.items[item + item_step]);
+                if (j + 2 >= ns && load_next) {
+                    load_q(a.items[next]);
+                    q_item = next;
+                }
             }
             if (!ok) break;
             g += ns;
@@ -485,7 +540,8 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                 }
             }
             dev::tc_fence_before();
-            dev::mbar_arrive(o_free);
+            if (had0) dev::mbar_arrive(&o_free[0]);
+            if (had1) dev::mbar_arrive(&o_free[1]);
             if (wg == 0 && row_valid)
                 a.part_lse[it.part_row0 + r] = (m + __log2f(l_tot)) * 0.69314718055994531f;
         }
