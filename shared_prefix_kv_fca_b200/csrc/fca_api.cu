@@ -131,20 +131,15 @@ fca_status fca_plan(const int32_t* block_tables, int32_t max_blocks, const int32
     return FCA_OK;
 }
 
-// SMs given to the grouped pass when it runs beside the per-request pass.
-// Rates per SM measured on B200 with both passes running: about 12.5 GB/s
-// of K/V streamed by the grouped pass (its per-head reads use an eighth of
-// each DRAM row, and its MMA/softmax pipeline runs at about that pace) and
-// 49 GB/s for the per-request pass.  The grouped pass streams a group's
-// tokens once per 128-row query tile, so its work is counted in tile-tokens.
-// It gets 0.9 of the SMs that would make both finish together; both passes
-// take their items from fixed or longest-first lists, and a sweep of fixed
-// splits on four workloads put this within a few percent of the best split.
-// Each pass is launched on its own SMs: run on every SM, the per-request
-// pass shares SMs with the grouped one and slows it.
+// SMs given to the grouped pass when it runs beside the per-request pass:
+// 0.9 of the share that would make both finish together at their measured
+// per-SM rates (kPrefixGBsPerSM, kSuffixGBsPerSM), the grouped pass's work
+// counted in tile-tokens.  A sweep of fixed splits on four workloads put this
+// next to the best split.  Each pass is launched on its own SMs: run on every
+// SM, the per-request pass shares SMs with the grouped one and slows it.
 static int prefix_share(const fca_plan_s* P, int sms) {
-    const double tp = (double)P->hdr.prefix_tile_tok_sum / 12.5;
-    const double ts = (double)P->hdr.suffix_tok_sum / 49.0;
+    const double tp = (double)P->hdr.prefix_tile_tok_sum / kPrefixGBsPerSM;
+    const double ts = (double)P->hdr.suffix_tok_sum / kSuffixGBsPerSM;
     const int n = (int)(0.9 * sms * tp / (tp + ts) + 0.5);
     return std::max(1, std::min(sms - 1, n));
 }

@@ -33,6 +33,13 @@ constexpr int32_t kErrStaticBlockId = 16;  // a used table entry outside [0, num
 // Size of the fixed device array behind fca_paged_decode_static.
 constexpr size_t kStaticScratchBytes = size_t(64) << 20;
 
+// Per-SM throughput of the two passes when they run side by side, measured on
+// B200 (K/V bytes a second per SM): the grouped pass streams a group's tokens
+// once per 128-row query tile, the per-request pass its own tokens.  Used to
+// split the SMs between the passes and to size the grouped pass's chunks.
+constexpr double kPrefixGBsPerSM = 18.0;
+constexpr double kSuffixGBsPerSM = 49.0;
+
 // Planner status bits (read back inside fca_plan).
 constexpr int32_t kPlanBadSeqLen = 1;
 constexpr int32_t kPlanBadBlockId = 2;

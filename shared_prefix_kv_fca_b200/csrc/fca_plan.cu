@@ -526,9 +526,8 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
     int32_t split_p = A.split_opt, split_s = A.split_opt;
     if (split_p <= 0) {
         // about three items per CTA of the grouped pass, which runs beside the
-        // per-request pass on its share of the SMs (the same estimate the
-        // decode uses: 12.5 GB/s per SM of tile-tokens against 49 for own tokens)
-        const double tp = (double)wp / 12.5, tsf = (double)ws / 49.0;
+        // per-request pass on its share of the SMs (the estimate the decode uses)
+        const double tp = (double)wp / kPrefixGBsPerSM, tsf = (double)ws / kSuffixGBsPerSM;
         const int32_t np = tp + tsf > 0.0 ? max(1, (int32_t)(0.9 * A.num_sms * tp / (tp + tsf) + 0.5)) : A.num_sms;
         const int64_t t = wp / (int64_t)(3 * min(max(1, A.num_sms), np));
         // no chunk above 4096 tokens: groups of very different lengths need

@@ -11,11 +11,13 @@
 // Work item = (group, KV head, 128-row Q tile, token chunk).  The kernel is
 // persistent: one CTA per SM walks its items (blockIdx.x, +gridDim.x, ...),
 // tensor memory is allocated once, and the K/V stream runs on across items.
-// 352 threads in four roles:
-//   warp 0      TMA producer: 64-token stages of K and V (four paged 16-token
-//               blocks, 64-column halves, 128-byte swizzle) into a ring of
-//               kPreStages slots; blocks past a chunk are loaded from rows
-//               beyond the cache, which TMA fills with zeros;
+// 384 threads in five roles:
+//   warps 0, 11 TMA producers, one for K and one for V: 64-token stages (four
+//               paged 16-token blocks, 64-column halves, 128-byte swizzle)
+//               into a ring of kPreStages slots; blocks past a chunk are
+//               loaded from rows beyond the cache, which TMA fills with
+//               zeros.  One issuing thread manages about one 2 KB box per
+//               hundred cycles, which alone would pace the pipeline;
 //   warps 2-9   two softmax warpgroups, one thread per query row each.  Stage
 //               s of an item belongs to warpgroup s % 2, which has its own S
 //               buffer, P buffer, O accumulator, copy of the Q tile and
@@ -61,8 +63,9 @@ namespace {
 
 constexpr int kPreStages = 5;
 constexpr int kSoftWarps = 8;
-constexpr int kPreThreads = 96 + kSoftWarps * 32;     // producer, MMA issuer 0, 8 softmax warps, MMA issuer 1
+constexpr int kPreThreads = 128 + kSoftWarps * 32;    // K producer, MMA issuer 0, 8 softmax warps, MMA issuer 1, V producer
 constexpr int kMmaWarp1 = 2 + kSoftWarps;             // the second MMA-issuing warp
+constexpr int kVWarp = 3 + kSoftWarps;                // the V producer
 constexpr float kRescaleLog2 = 8.f;
 
 struct PrefixArgs {
@@ -165,20 +168,23 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     dev::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        // The whole warp fetches block ids, 32 at a time (eight stages' worth)
-        // and one batch ahead, so no table lookup sits on the issue path;
-        // lane 0 waits for free slots and issues the copies.
+    if (warp == 0 || warp == kVWarp) {
+        // ------------------------------------------------ TMA producers
+        // One warp streams K, another V: a single thread issues a TMA box
+        // about every hundred cycles, which alone would pace the pipeline.
+        // Each warp fetches block ids, 32 at a time (eight stages' worth) and
+        // one batch ahead, so no table lookup sits on the issue path; lane 0
+        // waits for free slots and issues the copies.
+        const bool is_k = warp == 0;
+        uint64_t* full = is_k ? k_full : v_full;
+        uint64_t* empty = is_k ? k_empty : v_empty;
+        const CUtensorMap* tm = is_k ? &tmK : &tmV;
+        uint8_t* const ring = smem + (is_k ? L::kOffK : L::kOffV);
         constexpr int kBlkPerStage = kStageTokens / kBlockSize;
         constexpr int kStagesPerBatch = 32 / kBlkPerStage;
-        if (lane == 0) {
-            dev::tma_prefetch_desc(&tmK);
-            dev::tma_prefetch_desc(&tmV);
-        }
+        if (lane == 0) dev::tma_prefetch_desc(tm);
         uint32_t g = 0;
         bool ok = true;
-        int32_t pending_k = -1;     // stage whose K copies are in flight but whose V is not issued
         for (int32_t item = first_item; ok && item < a.n_items; item += item_step) {
             const PrefixItem it = a.items[item];
             const int32_t* row = a.bt + (int64_t)it.bt_row * a.max_blocks;
@@ -190,7 +196,7 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                 return blk < blk_end ? __ldg(row + blk) * kBlockSize : a.num_blocks * kBlockSize;
             };
             int32_t nxt = fetch(0), cur = 0;
-            for (int32_t j = 0; j < ns; ++j, ++g) {
+            for (int32_t j = 0; j < ns; ++j) {
                 if (j % kStagesPerBatch == 0) {
                     cur = nxt;
                     nxt = fetch(j / kStagesPerBatch + 1);
@@ -201,47 +207,29 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                     trow[bi] = __shfl_sync(0xffffffffu, cur, (j % kStagesPerBatch) * kBlkPerStage + bi);
                 if (lane == 0) {
                     const int s = g % kPreStages;
-                    const uint32_t ph = ((g / kPreStages) - 1) & 1;
-                    uint8_t* kdst = smem + L::kOffK + s * L::kKV;
-                    uint8_t* vdst = smem + L::kOffV + s * L::kKV;
-                    if (g >= kPreStages && !dev::mbar_wait(&k_empty[s], ph, abort_flag, a.err)) {
+                    uint8_t* dst = ring + s * L::kKV;
+                    if (g >= kPreStages && !dev::mbar_wait(&empty[s], ((g / kPreStages) - 1) & 1, abort_flag, a.err)) {
                         ok = false;
                     } else {
-                        dev::mbar_arrive_expect_tx(&k_full[s], L::kKV);
+                        dev::mbar_arrive_expect_tx(&full[s], L::kKV);
 #pragma unroll
                         for (int bi = 0; bi < kBlkPerStage; ++bi)
 #pragma unroll
                             for (int hf = 0; hf < L::kHalves; ++hf)
-                                dev::tma_load_3d(kdst + hf * (64 * 128) + bi * 2048, &tmK, &k_full[s], hf * 64,
-                                                 it.head, trow[bi]);
-                        pending_k = (int32_t)g;
-                        if (g >= kPreStages && !dev::mbar_wait(&v_empty[s], ph, abort_flag, a.err)) {
-                            ok = false;
-                        } else {
-                            dev::mbar_arrive_expect_tx(&v_full[s], L::kKV);
-#pragma unroll
-                            for (int bi = 0; bi < kBlkPerStage; ++bi)
-#pragma unroll
-                                for (int hf = 0; hf < L::kHalves; ++hf)
-                                    dev::tma_load_3d(vdst + hf * (64 * 128) + bi * 2048, &tmV, &v_full[s], hf * 64,
-                                                     it.head, trow[bi]);
-                            pending_k = -1;
-                        }
+                                dev::tma_load_3d(dst + hf * (64 * 128) + bi * 2048, tm, &full[s], hf * 64, it.head,
+                                                 trow[bi]);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
+                ++g;
             }
         }
         if (lane == 0) {
-            // never leave with copies in flight
+            // never leave with copies in flight (each slot's latest use only)
             volatile int never = 0;
-            if (pending_k >= 0)
-                dev::mbar_wait(&k_full[pending_k % kPreStages], (pending_k / kPreStages) & 1, &never, a.err);
-            for (uint32_t j = g; j > 0 && j + kPreStages > g; --j) {
-                dev::mbar_wait(&k_full[(j - 1) % kPreStages], ((j - 1) / kPreStages) & 1, &never, a.err);
-                dev::mbar_wait(&v_full[(j - 1) % kPreStages], ((j - 1) / kPreStages) & 1, &never, a.err);
-            }
+            for (uint32_t j = g; j > 0 && j + kPreStages > g; --j)
+                dev::mbar_wait(&full[(j - 1) % kPreStages], ((j - 1) / kPreStages) & 1, &never, a.err);
         }
         __syncwarp();
     } else if (warp == 1 || warp == kMmaWarp1) {
