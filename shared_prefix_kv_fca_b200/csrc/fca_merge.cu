@@ -6,13 +6,26 @@
 // partials are, in order, every split chunk of every group on r's chain and
 // every split chunk of r's own pass:
 //     lse = log(sum_i exp(lse_i)),   out = sum_i exp(lse_i - lse) * o_i,
-// with o_i already normalised by its own softmax sum.  One warp per
-// (r, hq).  The partials are taken 32 at a time: lane i finds the row of
-// partial i of the batch and reads its lse, one shuffle reduction gives the
-// batch maximum and weight sum (the running state is rescaled when the
-// maximum grows), then the o rows stream in four at a time, each lane owning
-// a contiguous slice of head_dim.  Partials with lse = -inf (empty chunks)
-// are skipped without reading their rows.
+// with o_i already normalised by its own softmax sum.
+//
+// Work unit: (request, KV head, slab of up to four of that KV head's query
+// heads), taken by W warps (W = 1, 2, 4 or 8, more when there are few units
+// and many partials per unit).  Every pass writes the G query heads of one
+// (request, KV head, chunk) as G consecutive partial rows, so a slab's rows of
+// one partial are one contiguous run of 4 x head_dim floats: each lane owns
+// float4 slots of that run, and the request's group chain is walked once per
+// slab, not once per query head.  The chain entries are read by one lane each
+// (all in parallel) and a warp scan turns their chunk counts into partial
+// offsets, so locating partial k costs shuffles rather than dependent loads.
+//
+// Warp w of a unit takes partials w, w + W, w + 2W, ... 32 at a time: lane i
+// locates partial i of the batch and reads its lse values; shuffle reductions
+// give each head's batch maximum and weight sum (the running state is
+// rescaled when a maximum grows); then the rows are accumulated two partials
+// at a time.  Partials with lse = -inf (empty chunks) never contribute.  With
+// W > 1 the warps' states (maximum, sum, accumulator) are combined through
+// shared memory.  A unit's warps share one CTA, so W > 1 only when units are
+// few (about 8 warps per SM in all) and each has many partials to read.
 #include <cuda_bf16.h>
 
 #include "fca_internal.h"
@@ -20,7 +33,7 @@
 namespace fca {
 
 struct MergeArgs {
-    int32_t R, Hq, G;
+    int32_t R, Hq, Hkv, G, n_slabs, W;
     const int32_t* chain_off;
     const int32_t* chain_g;
     const int32_t* chain_pos;
@@ -37,110 +50,249 @@ struct MergeArgs {
 
 namespace {
 
+constexpr int kSlabHeads = 4;   // query heads per unit
+constexpr int kWarps = 8;       // warps per CTA
+constexpr unsigned kFull = 0xffffffffu;
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
     return v;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
     return v;
 }
 
-template <int V>
-__device__ __forceinline__ void load_row(const float* src, float (&o)[V]) {
-    if constexpr (V == 4) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(src));
-        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-    } else {
-        const float2 v = __ldg(reinterpret_cast<const float2*>(src));
-        o[0] = v.x; o[1] = v.y;
+__device__ __forceinline__ int32_t warp_incl_scan(int32_t v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t u = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) v += u;
     }
+    return v;
 }
+
+// a[i] for a lane-dependent i, without indexing a register array at run time
+__device__ __forceinline__ float pick(const float (&a)[kSlabHeads], int i) {
+    float r = a[0];
+#pragma unroll
+    for (int k = 1; k < kSlabHeads; ++k) r = (i == k) ? a[k] : r;
+    return r;
+}
+
+template <int D>
+struct MergeSmem {
+    static constexpr int kSlots = kSlabHeads * D / 128;
+    float4 acc[kWarps][kSlots][32];
+    float m[kWarps][kSlabHeads];
+    float l[kWarps][kSlabHeads];
+};
 
 }  // namespace
 
 template <int D>
-__global__ void __launch_bounds__(256) k_merge(MergeArgs a) {
-    constexpr int V = D / 32;   // floats per lane
-    constexpr int kInFlight = 4;
+__global__ void __launch_bounds__(256, 3) k_merge(MergeArgs a) {
+    constexpr int kSlots = kSlabHeads * D / 128;   // float4 slots per lane
+    constexpr int kInFlight = 2;                    // partials loaded together
+    __shared__ MergeSmem<D> sm;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t pair = (int64_t)blockIdx.x * 8 + warp;
-    if (pair >= (int64_t)a.R * a.Hq) return;
-    const int32_t r = (int32_t)(pair / a.Hq), hq = (int32_t)(pair % a.Hq);
-    const int32_t h = hq / a.G, gq = hq % a.G;
-    const int32_t c0 = a.chain_off[r], c1 = a.chain_off[r + 1];
-    const int32_t nsc = a.s_nch[r];
-    int32_t n = nsc;
-    for (int32_t c = c0; c < c1; ++c) n += a.g_nch[a.chain_g[c]];
+    const int W = a.W, sub = warp % W;
+    const int64_t unit = (int64_t)blockIdx.x * (kWarps / W) + warp / W;
+    const bool active = unit < (int64_t)a.R * a.Hkv * a.n_slabs;   // uniform across a unit's warps
+    const int32_t slab = active ? (int32_t)(unit % a.n_slabs) : 0;
+    const int32_t rh = active ? (int32_t)(unit / a.n_slabs) : 0;
+    const int32_t r = rh / a.Hkv, h = rh % a.Hkv;
+    const int32_t gq0 = slab * kSlabHeads;
+    const int32_t nh = min(kSlabHeads, a.G - gq0);   // valid heads of this slab
 
-    // row of partial k of this pair (-1 past the end)
-    auto partial_row = [&](int32_t k) -> int32_t {
-        for (int32_t c = c0; c < c1; ++c) {
-            const int32_t g = a.chain_g[c], nch = a.g_nch[g];
-            if (k < nch) return a.g_part[g] + ((h * nch + k) * a.g_nm[g] + a.chain_pos[c]) * a.G + gq;
-            k -= nch;
+    // slot j of this lane: float index f = j * 128 + lane * 4 of the slab's run
+    int slot_head[kSlots];
+#pragma unroll
+    for (int j = 0; j < kSlots; ++j) slot_head[j] = (j * 128 + lane * 4) / D;
+
+    float m[kSlabHeads], l[kSlabHeads];
+#pragma unroll
+    for (int i = 0; i < kSlabHeads; ++i) { m[i] = -INFINITY; l[i] = 0.f; }
+    float4 acc[kSlots];
+#pragma unroll
+    for (int j = 0; j < kSlots; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+
+    if (active) {
+        // ---- the request's partials: chain entries (one lane each), then its own chunks
+        const int32_t c0 = a.chain_off[r], depth = a.chain_off[r + 1] - c0;
+        const int32_t nsc = a.s_nch[r], spart = a.s_part[r];
+        const bool wide = depth < 32;   // warp-uniform: every entry fits one lane
+        int32_t e_nch = 0, e_base = 0, e_step = 0;
+        if (wide) {
+            // entry e < depth: group chain[e]; row of (chunk k, slab) =
+            //   g_part + ((h nch + k) nm + pos) G + gq0 = e_base + k * e_step
+            // entry depth: own chunks, row = s_part + (h nsc + k) G + gq0
+            if (lane < depth) {
+                const int32_t g = a.chain_g[c0 + lane], pos = a.chain_pos[c0 + lane];
+                const int32_t nch = a.g_nch[g], nm = a.g_nm[g];
+                e_nch = nch;
+                e_base = a.g_part[g] + ((h * nch) * nm + pos) * a.G + gq0;
+                e_step = nm * a.G;
+            } else if (lane == depth) {
+                e_nch = nsc;
+                e_base = spart + h * nsc * a.G + gq0;
+                e_step = a.G;
+            }
         }
-        return k < nsc ? a.s_part[r] + (h * nsc + k) * a.G + gq : -1;
-    };
+        const int32_t e_end = warp_incl_scan(e_nch, lane);   // exclusive end of entry's partials
+        int32_t n = nsc;
+        if (wide) {
+            n = __shfl_sync(kFull, e_end, depth);
+        } else {
+            for (int32_t c = c0; c < c0 + depth; ++c) n += a.g_nch[a.chain_g[c]];
+        }
 
-    float m = -INFINITY, l = 0.f;
-    float acc[V];
-#pragma unroll
-    for (int i = 0; i < V; ++i) acc[i] = 0.f;
-
-    for (int32_t b0 = 0; b0 < n; b0 += 32) {
-        const int32_t row = partial_row(b0 + lane);
-        const float li = row >= 0 ? __ldg(a.part_lse + row) : -INFINITY;
-        const float mb = warp_max(li);
-        if (mb == -INFINITY) continue;              // every partial of the batch is empty
-        const float m_new = fmaxf(m, mb);
-        const float sc = expf(m - m_new);           // 0 while nothing has been added
-        l *= sc;
-#pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] *= sc;
-        const float wi = li == -INFINITY ? 0.f : expf(li - m_new);
-        l += warp_sum(wi);
-        m = m_new;
-        const int32_t nb = min(32, n - b0);
-        for (int32_t j0 = 0; j0 < nb; j0 += kInFlight) {
-            float o[kInFlight][V], w[kInFlight];
-#pragma unroll
-            for (int u = 0; u < kInFlight; ++u) {
-                const int32_t j = j0 + u;
-                const int32_t rj = __shfl_sync(0xffffffffu, row, j & 31);
-                w[u] = __shfl_sync(0xffffffffu, wi, j & 31);
-                if (j >= nb) w[u] = 0.f;
-                if (w[u] > 0.f) {
-                    load_row<V>(a.part_o + (int64_t)rj * D + lane * V, o[u]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < V; ++i) o[u][i] = 0.f;
+        const int32_t n_mine = n > sub ? (n - sub + W - 1) / W : 0;   // partials sub, sub + W, ...
+        for (int32_t b0 = 0; b0 < n_mine; b0 += 32) {
+            // row of the slab's first head in partial k of the request (-1 past the end)
+            int32_t row = -1;
+            int32_t k = (b0 + lane) * W + sub;
+            if (wide) {
+                int32_t e = 0;
+                for (int32_t i = 0; i < depth; ++i) e += (k >= __shfl_sync(kFull, e_end, i)) ? 1 : 0;
+                const int32_t end = __shfl_sync(kFull, e_end, e);
+                const int32_t cnt = __shfl_sync(kFull, e_nch, e);
+                const int32_t base = __shfl_sync(kFull, e_base, e);
+                const int32_t step = __shfl_sync(kFull, e_step, e);
+                if (k < n) row = base + (k - (end - cnt)) * step;
+            } else if (k < n) {
+                for (int32_t c = c0; c < c0 + depth && row < 0; ++c) {
+                    const int32_t g = a.chain_g[c], nch = a.g_nch[g];
+                    if (k < nch) row = a.g_part[g] + ((h * nch + k) * a.g_nm[g] + a.chain_pos[c]) * a.G + gq0;
+                    k -= nch;
                 }
+                if (row < 0) row = spart + (h * nsc + k) * a.G + gq0;
+            }
+            float li[kSlabHeads], wi[kSlabHeads], sc[kSlabHeads];
+#pragma unroll
+            for (int i = 0; i < kSlabHeads; ++i)
+                li[i] = (row >= 0 && i < nh) ? __ldg(a.part_lse + row + i) : -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kSlabHeads; ++i) {
+                const float m_new = fmaxf(m[i], warp_max(li[i]));
+                sc[i] = m_new == -INFINITY ? 1.f : expf(m[i] - m_new);   // 0 while nothing has been added
+                wi[i] = li[i] == -INFINITY ? 0.f : expf(li[i] - m_new);
+                l[i] = l[i] * sc[i] + warp_sum(wi[i]);
+                m[i] = m_new;
             }
 #pragma unroll
-            for (int u = 0; u < kInFlight; ++u)
+            for (int j = 0; j < kSlots; ++j) {
+                const float s = pick(sc, slot_head[j]);
+                acc[j].x *= s; acc[j].y *= s; acc[j].z *= s; acc[j].w *= s;
+            }
+            const int32_t nb = min(32, n_mine - b0);
+            for (int32_t j0 = 0; j0 < nb; j0 += kInFlight) {
+                float4 o[kInFlight][kSlots];
+                float w[kInFlight][kSlots];
 #pragma unroll
-                for (int i = 0; i < V; ++i) acc[i] = fmaf(w[u], o[u][i], acc[i]);
+                for (int u = 0; u < kInFlight; ++u) {
+                    const int32_t jj = (j0 + u) & 31;
+                    const int32_t rj = __shfl_sync(kFull, row, jj);
+                    float wh[kSlabHeads];
+#pragma unroll
+                    for (int i = 0; i < kSlabHeads; ++i) wh[i] = __shfl_sync(kFull, wi[i], jj);
+                    const float* src = a.part_o + (int64_t)rj * D + lane * 4;
+#pragma unroll
+                    for (int j = 0; j < kSlots; ++j) {
+                        w[u][j] = (j0 + u < nb && slot_head[j] < nh) ? pick(wh, slot_head[j]) : 0.f;
+                        o[u][j] = w[u][j] > 0.f ? __ldg(reinterpret_cast<const float4*>(src + j * 128))
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kInFlight; ++u)
+#pragma unroll
+                    for (int j = 0; j < kSlots; ++j) {
+                        acc[j].x = fmaf(w[u][j], o[u][j].x, acc[j].x);
+                        acc[j].y = fmaf(w[u][j], o[u][j].y, acc[j].y);
+                        acc[j].z = fmaf(w[u][j], o[u][j].z, acc[j].z);
+                        acc[j].w = fmaf(w[u][j], o[u][j].w, acc[j].w);
+                    }
+            }
         }
     }
 
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* dst = a.out + pair * D + lane * V;
+    // ---- combine the W warps of a unit (W is uniform across the CTA)
+    if (W > 1) {
 #pragma unroll
-    for (int i = 0; i < V; i += 2) {
-        *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+        for (int j = 0; j < kSlots; ++j) sm.acc[warp][j][lane] = acc[j];
+        if (lane < kSlabHeads) {
+            sm.m[warp][lane] = pick(m, lane);
+            sm.l[warp][lane] = pick(l, lane);
+        }
+        __syncthreads();
+        if (sub != 0) return;
+#pragma unroll
+        for (int i = 0; i < kSlabHeads; ++i) {
+            float mm = -INFINITY;
+            for (int v = 0; v < W; ++v) mm = fmaxf(mm, sm.m[warp + v][i]);
+            float ll = 0.f;
+            for (int v = 0; v < W; ++v) {
+                const float mv = sm.m[warp + v][i];
+                ll += mv == -INFINITY ? 0.f : sm.l[warp + v][i] * expf(mv - mm);
+            }
+            m[i] = mm;
+            l[i] = ll;
+        }
+#pragma unroll
+        for (int j = 0; j < kSlots; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int v = 0; v < W; ++v) {
+            float f[kSlabHeads];
+#pragma unroll
+            for (int i = 0; i < kSlabHeads; ++i) {
+                const float mv = sm.m[warp + v][i];
+                f[i] = mv == -INFINITY ? 0.f : expf(mv - m[i]);
+            }
+#pragma unroll
+            for (int j = 0; j < kSlots; ++j) {
+                const float s = pick(f, slot_head[j]);
+                const float4 x = sm.acc[warp + v][j][lane];
+                acc[j].x = fmaf(s, x.x, acc[j].x);
+                acc[j].y = fmaf(s, x.y, acc[j].y);
+                acc[j].z = fmaf(s, x.z, acc[j].z);
+                acc[j].w = fmaf(s, x.w, acc[j].w);
+            }
+        }
     }
-    if (a.lse && lane == 0) a.lse[pair] = l > 0.f ? m + logf(l) : -INFINITY;
+    if (!active) return;
+
+    // ---- normalise and store: out[r][h G + gq0 + head][col], lse[r][h G + gq0 + head]
+    float inv[kSlabHeads];
+#pragma unroll
+    for (int i = 0; i < kSlabHeads; ++i) inv[i] = l[i] > 0.f ? 1.f / l[i] : 0.f;
+    const int64_t q0 = (int64_t)r * a.Hq + (int64_t)h * a.G + gq0;   // first query head of the slab
+#pragma unroll
+    for (int j = 0; j < kSlots; ++j) {
+        if (slot_head[j] >= nh) continue;
+        const float s = pick(inv, slot_head[j]);
+        uint2 v;
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j].x * s, acc[j].y * s);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j].z * s, acc[j].w * s);
+        v.x = *reinterpret_cast<uint32_t*>(&lo);
+        v.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(a.out + q0 * D + j * 128 + lane * 4) = v;
+    }
+    if (a.lse && lane < nh) {
+        const float mm = pick(m, lane), ll = pick(l, lane);
+        a.lse[q0 + lane] = ll > 0.f ? mm + logf(ll) : -INFINITY;
+    }
 }
 
 cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, cudaStream_t stream) {
     MergeArgs a;
     a.R = P->R;
     a.Hq = P->Hq;
+    a.Hkv = P->Hkv;
     a.G = P->G;
+    a.n_slabs = (P->G + kSlabHeads - 1) / kSlabHeads;
     a.chain_off = P->chain_off;
     a.chain_g = P->chain_g;
     a.chain_pos = P->chain_pos;
@@ -153,12 +305,27 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, cudaStream_
     a.part_lse = P->part_lse;
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
+    const int64_t units = (int64_t)P->R * P->Hkv * a.n_slabs;
+    // Warps per unit: split a unit's partials over more warps only while the
+    // whole grid stays under about 8 warps per SM and every warp still gets
+    // two partials or more on average (a sweep of 8, 16 and 32 warps per SM on
+    // the four large workloads favoured 8: extra warps per unit cost more in
+    // the combine than they save when units are plentiful).
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t pairs = (int64_t)P->R * P->Hq;
-    const int grid = (int)((pairs + 7) / 8);
+    const int64_t n_part = (int64_t)P->hdr.n_prefix_partials + P->hdr.n_suffix_partials;
+    const double per_pair = pairs > 0 ? (double)n_part / (double)pairs : 0.0;
+    int W = 1;
+    while (W < kWarps && units * W < (int64_t)sms * 8 && 2.0 * W <= per_pair) W *= 2;
+    a.W = W;
+    const int64_t per_cta = kWarps / W;
+    const int grid = (int)((units + per_cta - 1) / per_cta);
+    if (grid == 0) return cudaSuccess;
     if (P->D == 128)
-        k_merge<128><<<grid, 256, 0, stream>>>(a);
+        k_merge<128><<<grid, 32 * kWarps, 0, stream>>>(a);
     else
-        k_merge<64><<<grid, 256, 0, stream>>>(a);
+        k_merge<64><<<grid, 32 * kWarps, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

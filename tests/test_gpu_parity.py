@@ -160,6 +160,24 @@ def test_decode_one_group_of_many_members():
     assert_close(o, l, o_ref, l_ref, "one wide group")
 
 
+@pytest.mark.parametrize("shape", [(8, 2, 128), (6, 2, 64)])
+def test_decode_deep_chain(shape):
+    # request j shares blocks 0..j with every request after it: one nested
+    # group per block, so the last requests sit under 30-40 groups (chains
+    # longer than a warp's 32 lanes take the merge's sequential walk)
+    Hq, Hkv, D = shape
+    rng = np.random.default_rng(31)
+    n = 42
+    reqs = [[(f"k{d}", 16) for d in range(j + 1)] + [(None, int(rng.integers(0, 24)))] for j in range(n)]
+    w = fca_workloads.fill("deep", reqs, Hq=Hq, Hkv=Hkv, D=D, seed=31, rng=rng, poison_padding=True)
+    o, l, exp, _ = run(w)
+    ref = oracle.plan(w.block_tables, w.seq_lens, w.block_size)
+    assert_plan_equal(exp, ref)
+    assert len(ref["a"]) >= 36
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(o, l, o_ref, l_ref, f"deep chain {shape}")
+
+
 @pytest.mark.parametrize("split", [64, 128, 256])
 def test_decode_small_splits(split):
     # many split chunks per group and per request, ragged tails
