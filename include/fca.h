@@ -116,7 +116,8 @@ fca_status fca_plan(const int32_t *block_tables, int32_t max_blocks, const int32
  *            16-byte aligned.
  *   out      DEVICE bf16 [num_requests][num_q_heads][head_dim] (round to nearest even).
  *   lse      DEVICE fp32 [num_requests][num_q_heads], or NULL to skip.
- *   scale    multiplier of q.k (normally 1/sqrt(head_dim)).
+ *   scale    multiplier of q.k (normally 1/sqrt(head_dim)); positive and finite,
+ *            else FCA_ERR_INVALID_ARG.
  *
  * Asynchronous on `stream`.  When the plan has both grouped and per-request
  * work, the two passes run side by side on disjoint sets of SMs: the grouped

@@ -147,6 +147,7 @@ static int prefix_share(const fca_plan_s* P, int sms) {
 static fca_status decode_impl(const void* q, const void* k_cache, const void* v_cache, fca_plan_t plan, void* out,
                               float* lse, float scale, void* stream) {
     if (!plan || !q || !k_cache || !v_cache || !out) return FCA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < INFINITY)) return FCA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return FCA_ERR_INVALID_ARG;
@@ -195,6 +196,7 @@ fca_status fca_decode(const void* q, const void* k_cache, const void* v_cache, f
 static fca_status pass_impl(int pass, const void* q, const void* k_cache, const void* v_cache, fca_plan_t plan,
                             float scale, void* stream) {
     if (!plan || !q || !k_cache || !v_cache) return FCA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < INFINITY)) return FCA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return FCA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     CUtensorMap tk, tv;

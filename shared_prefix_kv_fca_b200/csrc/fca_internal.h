@@ -46,11 +46,12 @@ constexpr int32_t kPlanBadBlockId = 2;
 constexpr int32_t kPlanInconsistent = 4;   // block ids do not identify prefixes
 constexpr int32_t kPlanTooManyGroups = 8;
 
-// One tile of the grouped prefix pass: rows [row0, row0 + nrows) of group
-// `group`'s stacked queries (member i / G, query head head * G + i % G),
-// against tokens [tok0, tok1) of the table row of request `bt_row`.
+// One tile of the grouped prefix pass: rows [row0, row0 + nrows) of a
+// group's stacked queries (member i / G, query head head * G + i % G; the
+// group's members start at members[moff]), against tokens [tok0, tok1) of the
+// table row of request `bt_row`.
 struct PrefixItem {
-    int32_t group, head, row0, nrows;
+    int32_t moff, head, row0, nrows;
     int32_t tok0, tok1, bt_row, part_row0;   // partial row of stacked row row0
 };
 

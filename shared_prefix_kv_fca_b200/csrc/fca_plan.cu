@@ -675,7 +675,7 @@ __global__ void k_fill_prefix_items(const PlanHeader* hdr, const int32_t* g_a, c
         for (int32_t i = threadIdx.x; i < Hkv * per_head; i += blockDim.x) {
             const int32_t h = i % Hkv, rem = i / Hkv, c = rem % nch, tile = rem / nch;
             PrefixItem it;
-            it.group = g;
+            it.moff = g_moff[g];
             it.head = h;
             it.row0 = tile * kPrefixTileRows;
             it.nrows = min(kPrefixTileRows, rows - it.row0);

@@ -30,8 +30,12 @@
 //               which after the first stages is rare (numerator and
 //               denominator use the same reference, so the result is exact).
 //               At the end of an item the two partial states are merged by
-//               their weights.  A group reloads its Q copy for its next item
-//               once it has read its own last S of the current one;
+//               their weights and the rows leave through the group's P buffer
+//               (coalesced 128-byte row segments).  A group reloads its Q copy
+//               for its next item once it has read its own last S of the
+//               current one; the request behind each of its rows is read when
+//               the current item starts, and the rows are prefetched into L2
+//               a few stages before the end;
 //   warps 1, 10 one MMA issuer per softmax group (warp 1 also allocates
 //               tensor memory): S = Q K^T (M=128, N=64, Q from tensor memory)
 //               and O_w += P V (M=128, N=head_dim, P from shared memory, the
@@ -67,13 +71,13 @@ constexpr int kPreThreads = 128 + kSoftWarps * 32;    // K producer, MMA issuer 
 constexpr int kMmaWarp1 = 2 + kSoftWarps;             // the second MMA-issuing warp
 constexpr int kVWarp = 3 + kSoftWarps;                // the V producer
 constexpr float kRescaleLog2 = 8.f;
+constexpr int kItemSlots = 64;      // items of a CTA kept in shared memory (later ones are read from global)
 
 struct PrefixArgs {
     const PrefixItem* items;
     int32_t n_items;
     const int32_t* bt;
     const int32_t* members;
-    const int32_t* g_moff;
     int32_t max_blocks, num_blocks, Hq, G;
     const __nv_bfloat16* q;
     float scale_log2;
@@ -95,7 +99,8 @@ struct PreLayout {
     // p_full[2], p_free[2], o_full[2], o_free[2], mma_done[2], l_bar
     static constexpr int kNumBars = 2 + 4 * kPreStages + 10 + 5;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kTotal = kOffMisc + 64 + 1024;   // + alignment slack
+    static constexpr int kOffItems = (kOffMisc + 64 + 15) / 16 * 16;   // this CTA's first kItemSlots items
+    static constexpr int kTotal = kOffItems + kItemSlots * (int)sizeof(PrefixItem) + 1024;   // + alignment slack
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0;                  // S of group w: 64 fp32 columns at 64 w
     static constexpr uint32_t kColO = 128;                // O of group w: D fp32 columns at 128 + D w
@@ -163,6 +168,17 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         dev::tmem_alloc(tmem_slot, L::kTmemCols);
         dev::tmem_relinquish();
     }
+    // The CTA's items (first_item, + item_step, ...) go to shared memory once,
+    // so that no role stalls on a global load when an item starts.
+    PrefixItem* items_s = reinterpret_cast<PrefixItem*>(smem + L::kOffItems);
+    {
+        const int32_t n_mine = first_item < a.n_items ? (a.n_items - first_item + item_step - 1) / item_step : 0;
+        for (int32_t k = threadIdx.x; k < min(n_mine, kItemSlots); k += blockDim.x)
+            items_s[k] = a.items[first_item + k * item_step];
+    }
+    auto item_at = [&](int32_t local, int32_t item) -> PrefixItem {
+        return local < kItemSlots ? items_s[local] : a.items[item];
+    };
     dev::tc_fence_before();
     __syncthreads();
     dev::tc_fence_after();
@@ -185,8 +201,9 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         if (lane == 0) dev::tma_prefetch_desc(tm);
         uint32_t g = 0;
         bool ok = true;
-        for (int32_t item = first_item; ok && item < a.n_items; item += item_step) {
-            const PrefixItem it = a.items[item];
+        int32_t local = 0;
+        for (int32_t item = first_item; ok && item < a.n_items; item += item_step, ++local) {
+            const PrefixItem it = item_at(local, item);
             const int32_t* row = a.bt + (int64_t)it.bt_row * a.max_blocks;
             const int32_t blk0 = it.tok0 / kBlockSize, blk_end = it.tok1 / kBlockSize;
             const int32_t ns = stages_of(it);
@@ -299,7 +316,7 @@ __global__ void __launch_bounds__(kPreThreads, 1)
             uint32_t g = 0;
             int32_t local = 0, q_items = 0;
             for (int32_t item = first_item; ok && item < a.n_items; item += item_step, ++local) {
-                const int32_t ns = stages_of(a.items[item]);
+                const int32_t ns = stages_of(item_at(local, item));
                 const int32_t j0 = ((g & 1) == (uint32_t)w) ? 0 : 1;
                 if (j0 < ns) {
                     // this group's Q copy holds the item's queries once q_full[w] completes
@@ -330,29 +347,36 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         const uint32_t s_col = L::kColS + wg * 64, o_col = L::kColO + wg * D;
         constexpr int kOHalf = D / 2;
 
+        // The request whose queries fill tile row r of an item: stacked row
+        // row0 + r is member (row0 + r) / G of the group.  Read when an item
+        // starts, for the next item, so that the load is long done when the
+        // row is needed.
+        auto member_of = [&](const PrefixItem& it) -> int32_t {
+            return r < it.nrows ? __ldg(a.members + it.moff + (it.row0 + r) / a.G) : 0;
+        };
+        auto q_row = [&](const PrefixItem& it, int32_t member) -> const uint4* {
+            const int32_t i = it.row0 + r;
+            return reinterpret_cast<const uint4*>(a.q + ((int64_t)member * a.Hq + it.head * a.G + i % a.G) * D);
+        };
         // Q tile row r (whole row): stacked row row0 + r = member (i / G),
         // query head head * G + i % G; rows past the tile are zero.
-        auto load_q = [&](const PrefixItem& it) {
+        auto load_q = [&](const PrefixItem& it, int32_t member) {
             const bool valid = r < it.nrows;
-            const uint4* src = nullptr;
-            if (valid) {
-                const int32_t i = it.row0 + r;
-                const int32_t member = a.members[a.g_moff[it.group] + i / a.G];
-                src = reinterpret_cast<const uint4*>(a.q + ((int64_t)member * a.Hq + it.head * a.G + i % a.G) * D);
-            }
+            const uint4* src = valid ? q_row(it, member) : nullptr;
+            // the whole row in one round trip, then the tensor-memory stores
+            uint32_t w[D / 64][32];
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-                uint32_t w[32];
+            for (int c = 0; c < D / 64; ++c)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const uint4 v = valid ? src[c * 8 + e] : make_uint4(0, 0, 0, 0);
-                    w[e * 4 + 0] = v.x;
-                    w[e * 4 + 1] = v.y;
-                    w[e * 4 + 2] = v.z;
-                    w[e * 4 + 3] = v.w;
+                    w[c][e * 4 + 0] = v.x;
+                    w[c][e * 4 + 1] = v.y;
+                    w[c][e * 4 + 2] = v.z;
+                    w[c][e * 4 + 3] = v.w;
                 }
-                dev::tmem_st32(tmem + lane_base + L::kColQ + wg * (D / 2) + c * 32, w);
-            }
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) dev::tmem_st32(tmem + lane_base + L::kColQ + wg * (D / 2) + c * 32, w[c]);
             dev::tc_wait_st();
             dev::tc_fence_before();
             dev::mbar_arrive(&q_full[wg]);
@@ -364,17 +388,20 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         uint32_t g = 0;
         int32_t local = 0;
         int32_t q_item = -1;                           // item whose queries this group's Q copy holds
+        int32_t member_cur = first_item < a.n_items ? member_of(item_at(0, first_item)) : 0;
         for (int32_t item = first_item; ok && item < a.n_items; item += item_step, ++local) {
-            const PrefixItem it = a.items[item];
+            const PrefixItem it = item_at(local, item);
             const int32_t ns = stages_of(it), n_tok = it.tok1 - it.tok0;
             const int32_t next = item + item_step;
+            const PrefixItem it_next = next < a.n_items ? item_at(local + 1, next) : it;
             // Q of the next item, if this group has stages there: loaded after the
             // group's last S of this item, when all of its Q K^T have completed
-            const bool load_next = next < a.n_items && has_stages(stages_of(a.items[next]), g + ns);
+            const bool load_next = next < a.n_items && has_stages(stages_of(it_next), g + ns);
+            const int32_t member_next = next < a.n_items ? member_of(it_next) : 0;
             // groups with stages in this item (their issuers wait for this epilogue)
             const bool had0 = (((g & 1) == 0u) ? 0 : 1) < ns, had1 = (((g & 1) == 1u) ? 0 : 1) < ns;
             if (has_stages(ns, g) && q_item != item) {
-                load_q(it);
+                load_q(it, member_cur);
                 q_item = item;
             }
             float m_ref = -INFINITY, l_run = 0.f;
@@ -399,21 +426,29 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                     }
                     dev::mbar_arrive(&p_full[wg]);
                     if (j + 2 >= ns && load_next) {
-                        load_q(a.items[next]);
+                        load_q(it_next, member_next);
                         q_item = next;
                     }
                     continue;
                 }
                 const int32_t n_valid = min(kStageTokens, n_tok - j * kStageTokens);
+                // raw scores q.k (both halves in flight together); the softmax
+                // scale is applied inside the exponent, as one FMA with the maximum
                 float x[64];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t t[32];
-                    dev::tmem_ld32(tmem + lane_base + s_col + h2 * 32, t);
+                {
+                    uint32_t t0[32], t1[32];
+                    dev::tmem_ld32(tmem + lane_base + s_col, t0);
+                    dev::tmem_ld32(tmem + lane_base + s_col + 32, t1);
                     dev::tc_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        x[h2 * 32 + i] = h2 * 32 + i < n_valid ? __uint_as_float(t[i]) * a.scale_log2 : -INFINITY;
+                    for (int i = 0; i < 32; ++i) {
+                        x[i] = __uint_as_float(t0[i]);
+                        x[32 + i] = __uint_as_float(t1[i]);
+                    }
+                }
+                if (n_valid < kStageTokens) {   // the chunk's last stage: tokens past it are masked
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) x[i] = i < n_valid ? x[i] : -INFINITY;
                 }
                 dev::tc_fence_before();
                 dev::mbar_arrive(&s_free[wg]);
@@ -422,8 +457,9 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                 for (int i = 0; i < 8; ++i) mx8[i] = x[i];
 #pragma unroll
                 for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], x[i]);
+                // the row maximum in the log2 domain (the scale is positive)
                 const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * a.scale_log2;
 
                 float alpha = 1.f;
                 bool rescale = false;
@@ -461,7 +497,8 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                 uint32_t pw[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float p0 = dev::ex2(x[2 * i] - m_ref), p1 = dev::ex2(x[2 * i + 1] - m_ref);
+                    const float p0 = dev::ex2(fmaf(x[2 * i], a.scale_log2, -m_ref));
+                    const float p1 = dev::ex2(fmaf(x[2 * i + 1], a.scale_log2, -m_ref));
                     ls[(2 * i) & 3] += p0;
                     ls[(2 * i + 1) & 3] += p1;
                     pw[i] = dev::pack_bf16x2(p0, p1);
@@ -476,12 +513,18 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                 dev::fence_proxy_async_smem();
                 dev::mbar_arrive(&p_full[wg]);
                 if (j + 2 >= ns && load_next) {
-                    load_q(a.items[next]);
+                    load_q(it_next, member_next);
                     q_item = next;
+                } else if (j + 2 < ns && j >= 2 && j < 4 && load_next && r < it_next.nrows) {
+                    // a stage before the end: start moving the next item's Q row into L2
+                    const uint4* src = q_row(it_next, member_next);
+                    dev::prefetch_l2(src);
+                    dev::prefetch_l2(reinterpret_cast<const uint8_t*>(src) + D);
                 }
             }
             if (!ok) break;
             g += ns;
+            member_cur = member_next;
 
             // epilogue: wait for this group's last P V, swap (m, l) with the other
             // group, and write half of the columns of the merged, normalised rows
@@ -506,14 +549,22 @@ __global__ void __launch_bounds__(kPreThreads, 1)
             const float l_tot = l0 * w0 + l1 * w1;
             const float inv = 1.f / l_tot, c0 = w0 * inv, c1 = w1 * inv;
             const bool row_valid = r < it.nrows;
-            float* dst = a.part_o + ((int64_t)it.part_row0 + r) * D + wg * kOHalf;
+            // The rows leave through this warp's quarter of the group's P buffer
+            // (free: the group's last P V has completed), 32 columns at a time, so
+            // that each global store writes four 128-byte row segments instead of
+            // 32 scattered 16-byte pieces.  Staging rows are 128 bytes, their
+            // 16-byte chunks swizzled by row so that both sides are conflict-free.
+            float* stage = reinterpret_cast<float*>(smem + L::kOffP + wg * 128 * 128 + quarter * 4096);
+            float* dst0 = a.part_o + ((int64_t)it.part_row0 + quarter * 32) * D + wg * kOHalf;
+#pragma unroll 1
+            for (int pass = 0; live && pass < kOHalf / 32; ++pass) {
 #pragma unroll
-            for (int c = 0; live && c < kOHalf / 16; ++c) {
-                uint32_t o0[16], o1[16];
-                dev::tmem_ld16(tmem + lane_base + L::kColO + wg * kOHalf + c * 16, o0);
-                dev::tmem_ld16(tmem + lane_base + L::kColO + D + wg * kOHalf + c * 16, o1);
-                dev::tc_wait_ld();
-                if (row_valid) {
+                for (int c = 0; c < 2; ++c) {
+                    const int col = wg * kOHalf + pass * 32 + c * 16;
+                    uint32_t o0[16], o1[16];
+                    dev::tmem_ld16(tmem + lane_base + L::kColO + col, o0);
+                    dev::tmem_ld16(tmem + lane_base + L::kColO + D + col, o1);
+                    dev::tc_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 16; i += 4) {
                         float v[4];
@@ -523,9 +574,20 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                             const float a1 = l1 > 0.f ? __uint_as_float(o1[i + e]) * c1 : 0.f;
                             v[e] = a0 + a1;
                         }
-                        *reinterpret_cast<float4*>(dst + c * 16 + i) = make_float4(v[0], v[1], v[2], v[3]);
+                        const int k = c * 4 + i / 4;
+                        *reinterpret_cast<float4*>(stage + lane * 32 + ((k ^ (lane & 7)) << 2)) =
+                            make_float4(v[0], v[1], v[2], v[3]);
                     }
                 }
+                __syncwarp();
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const int rr = t * 4 + (lane >> 3), k = lane & 7;
+                    const float4 v = *reinterpret_cast<const float4*>(stage + rr * 32 + ((k ^ (rr & 7)) << 2));
+                    if (quarter * 32 + rr < it.nrows)
+                        *reinterpret_cast<float4*>(dst0 + (int64_t)rr * D + pass * 32 + k * 4) = v;
+                }
+                __syncwarp();
             }
             dev::tc_fence_before();
             if (had0) dev::mbar_arrive(&o_free[0]);
@@ -569,7 +631,6 @@ cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const CUtensorMap&
     a.n_items = n;
     a.bt = P->bt;
     a.members = P->members;
-    a.g_moff = P->g_moff;
     a.max_blocks = P->max_blocks;
     a.num_blocks = P->num_blocks;
     a.Hq = P->Hq;

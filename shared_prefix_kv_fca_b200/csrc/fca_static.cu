@@ -140,7 +140,8 @@ extern "C" fca_status fca_paged_decode_static(const void* q, const void* k_cache
                                               int32_t head_dim, void* out, float* lse, float scale,
                                               int32_t* dev_status, void* stream) {
     if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !out || num_requests < 0 || max_blocks < 1 ||
-        num_blocks < 1 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads != 0)
+        num_blocks < 1 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads != 0 ||
+        !(scale > 0.f) || !(scale < INFINITY))
         return FCA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||

@@ -346,6 +346,11 @@ def test_error_paths_return_status():
     with fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D) as plan:
         with pytest.raises(fca.FcaError):
             fca.fca_flat_decode(q, k, v, plan, torch.empty_like(q))
+        # the scale must be positive and finite
+        for bad_scale in (0.0, -0.125, float("inf"), float("nan")):
+            with pytest.raises(fca.FcaError) as e:
+                fca.fca_decode(q, k, v, plan, torch.empty_like(q), None, bad_scale)
+            assert e.value.status == 1
         # the good plan still works after the failed calls
         out = torch.empty_like(q)
         fca.fca_decode(q, k, v, plan, out)
