@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
     }
     if (split_s <= 0) {
         const int64_t t = ws / (int64_t)(32 * max(1, A.num_sms));
-        split_s = (int32_t)min((int64_t)8192, max((int64_t)256, (t + 63) / 64 * 64));
+        split_s = (int32_t)min((int64_t)8192, max((int64_t)kMinOwnChunk, (t + 63) / 64 * 64));
     }
 
     // per-group chunk counts, item offsets, partial bases, member offsets

@@ -102,10 +102,25 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
         const int32_t nblk = (it.tok1 + kBlockSize - 1) / kBlockSize - blk0;
         const int32_t* row = a.bt + (int64_t)it.request * a.max_blocks + blk0;
 
-        auto issue = [&](int32_t j) {   // lane 0: block j of the item into its slot
+        // Block ids in registers, 32 at a time: lane l holds block 32 b + l of
+        // batch b (the current batch and the next; the next is read when the
+        // current one starts, long before it is needed), so no table lookup
+        // sits on lane 0's issue path.
+        auto bid_load = [&](int32_t b) -> int32_t {
+            const int32_t jj = b * 32 + lane;
+            return jj < nblk ? __ldg(row + jj) : 0;
+        };
+        int32_t bid_cur = bid_load(0), bid_nxt = nblk > 32 ? bid_load(1) : 0;
+        // id of block jj, which lies in batch `base` or the one after (all lanes call)
+        auto bid_of = [&](int32_t jj, int32_t base) -> int32_t {
+            const int32_t vc = __shfl_sync(0xffffffffu, bid_cur, jj & 31);
+            const int32_t vn = __shfl_sync(0xffffffffu, bid_nxt, jj & 31);
+            return (jj >> 5) == base ? vc : vn;
+        };
+        auto issue = [&](int32_t j, int32_t bid) {   // lane 0: block j of the item into its slot
             const uint32_t u = uses + j;
             const int s = u % L::kSlots;
-            const int32_t trow = row[j] * kBlockSize;
+            const int32_t trow = bid * kBlockSize;
             uint8_t* kdst = ring + s * L::kSlot;
             dev::fence_proxy_async_smem();
             dev::mbar_arrive_expect_tx(&full[s], L::kSlot);
@@ -115,8 +130,11 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
                 dev::tma_load_3d(kdst + L::kTile + hf * 2048, &tmV, &full[s], hf * 64, it.head, trow);
             }
         };
-        if (lane == 0)
-            for (int32_t j = 0; j < nblk && j < L::kSlots; ++j) issue(j);
+#pragma unroll
+        for (int32_t j = 0; j < L::kSlots; ++j) {
+            const int32_t bid = bid_of(j, 0);
+            if (lane == 0 && j < nblk) issue(j, bid);
+        }
 
         // Q^T fragments (B operand): column n = query head nt * 8 + g8,
         // rows k = head_dim pairs 16 ks + 2 tig (+8).  Heads past G are zero.
@@ -220,7 +238,13 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
                 for (int nt = 0; nt < NT; ++nt) dev::mma_bf16_16816(o[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
             }
             __syncwarp();
-            if (lane == 0 && j + L::kSlots < nblk) issue(j + L::kSlots);
+            if (((j + 1) & 31) == 0) {   // the next block starts a new batch of ids
+                bid_cur = bid_nxt;
+                bid_nxt = bid_load(((j + 1) >> 5) + 1);
+            }
+            const int32_t t = j + 1 + L::kSlots - 1;   // the block that takes the slot just freed
+            const int32_t bid_t = bid_of(t, (j + 1) >> 5);
+            if (lane == 0 && t < nblk) issue(t, bid_t);
         }
         uses += nblk;
         if (failed) break;
