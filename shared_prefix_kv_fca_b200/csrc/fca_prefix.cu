@@ -515,8 +515,9 @@ __global__ void __launch_bounds__(kPreThreads, 1)
                 if (j + 2 >= ns && load_next) {
                     load_q(it_next, member_next);
                     q_item = next;
-                } else if (j + 2 < ns && j >= 2 && j < 4 && load_next && r < it_next.nrows) {
-                    // a stage before the end: start moving the next item's Q row into L2
+                } else if (j >= ns - 8 && j < ns - 6 && load_next && r < it_next.nrows) {
+                    // this group's stage three before its last: start moving the next
+                    // item's Q row into L2 (earlier, and the KV stream evicts it again)
                     const uint4* src = q_row(it_next, member_next);
                     dev::prefetch_l2(src);
                     dev::prefetch_l2(reinterpret_cast<const uint8_t*>(src) + D);
