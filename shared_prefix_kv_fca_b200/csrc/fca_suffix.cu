@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
                 bid_cur = bid_nxt;
                 bid_nxt = bid_load(((j + 1) >> 5) + 1);
             }
-            const int32_t t = j + 1 + L::kSlots - 1;   // the block that takes the slot just freed
+            const int32_t t = j + L::kSlots;   // the block that takes the slot just freed
             const int32_t bid_t = bid_of(t, (j + 1) >> 5);
             if (lane == 0 && t < nblk) issue(t, bid_t);
         }
