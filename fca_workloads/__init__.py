@@ -35,6 +35,10 @@ Named configurations (one layer's decode step each):
                  until they sum to 1024 (last one cut); prompt lengths
                  log-uniform in [128, 16384] tokens, integer, not block
                  aligned; own U{1..2048}; 32/8/128.
+* ``pairs``      R=1024 = 512 pairs of requests, each pair on its own prompt
+                 of U{16..256} tokens; own U{256..1024}; 32/8/128.  Not one of
+                 the task's configurations: the low-sharing case that the
+                 planner's automatic folding of small groups is for.
 """
 from __future__ import annotations
 
@@ -60,6 +64,7 @@ CONFIGS = {
     "longctx": dict(Hq=32, Hkv=8, D=128),
     "forest": dict(Hq=64, Hkv=8, D=128),
     "mixed": dict(Hq=32, Hkv=8, D=128),
+    "pairs": dict(Hq=32, Hkv=8, D=128),
 }
 
 
@@ -302,6 +307,15 @@ def make(name: str, seed: int = 0, poison_padding: bool = False,
                 reqs.append([(key, plen), (None, int(rng.integers(1, 2049)))])
         desc = (f"1024 requests in {len(sizes)} groups (Zipf 1.2 on 1..64), prompts "
                 "log-U[128,16384] tokens, own U{1..2048}")
+        return fill(name, reqs, seed=seed, rng=rng, poison_padding=poison_padding,
+                    description=desc, **c)
+    if name == "pairs":
+        # the case sharing barely pays for: many pairs of requests on short prompts
+        for p in range(prompts or 512):
+            plen = int(rng.integers(16, 257))
+            for _ in range(2):
+                reqs.append([(f"p{p}", plen), (None, int(rng.integers(256, 1025)))])
+        desc = "512 pairs of requests, prompts U{16..256} tokens, own U{256..1024}"
         return fill(name, reqs, seed=seed, rng=rng, poison_padding=poison_padding,
                     description=desc, **c)
     raise KeyError(name)

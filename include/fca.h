@@ -69,13 +69,21 @@ typedef struct fca_plan_opts {
     int32_t split_tokens;      /* split-KV chunk length in tokens, multiple of 64;
                                   0 = automatic */
     int32_t flags;             /* FCA_PLAN_* bits */
+    int32_t min_saved_blocks;  /* a group is used only if (members - 1) x its length in
+                                  blocks -- the block reads sharing it saves -- reaches
+                                  this; otherwise it is folded like a short group
+                                  (>= 0; default 32, 0 = use every shared prefix).  The
+                                  automatic activation of "Core Mechanism": groups too
+                                  small to pay for their own grouped-pass work are
+                                  read by their members' own passes instead. */
 } fca_plan_opts;
 
 /* Build a plan with no groups: every request reads its whole table in its own
  * pass.  fca_decode on such a plan is the flat (non-cascaded) paged decode. */
 #define FCA_PLAN_FLAT 1u
 
-/* Default options (min_group_size 2, min_shared_blocks 1, split auto, flags 0). */
+/* Default options (min_group_size 2, min_shared_blocks 1, split auto, flags 0,
+ * min_saved_blocks 32). */
 void fca_plan_opts_default(fca_plan_opts *opts /* HOST, out */);
 
 /*

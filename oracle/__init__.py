@@ -63,8 +63,8 @@ def _load():
         lib.oracle_paged_attention.restype = ctypes.c_int
         lib.oracle_plan.argtypes = [
             i32p, ctypes.c_int32, ctypes.c_int32, i32p, ctypes.c_int32, ctypes.c_int32,
-            ctypes.c_int32, i32p, i32p, i32p, i32p, i32p, i32p, i32p, i32p, ctypes.c_int32,
-            ctypes.c_int64]
+            ctypes.c_int32, ctypes.c_int32, i32p, i32p, i32p, i32p, i32p, i32p, i32p, i32p,
+            ctypes.c_int32, ctypes.c_int64]
         lib.oracle_plan.restype = ctypes.c_int
         lib.oracle_unique_kv_tokens.argtypes = [i32p, ctypes.c_int32, ctypes.c_int32, i32p,
                                                 ctypes.c_int32, ctypes.c_int64]
@@ -145,8 +145,12 @@ def paged_attention(q, k_cache, v_cache, block_tables, seq_lens, scale: float, p
 
 
 def plan(block_tables, seq_lens, block_size: int, min_group_size: int = 2,
-         min_shared_blocks: int = 1) -> dict:
+         min_shared_blocks: int = 1, min_saved_blocks: int = 0) -> dict:
     """Canonical FCA plan from the naive trie.
+
+    min_saved_blocks: a group is kept only if (members - 1) x its length in
+    blocks reaches this (0 keeps every shared prefix; the CUDA planner's
+    default is 32).
 
     Returns dict with int32 arrays: a, b, parent, member_off, n_members (one
     entry per group, canonical order), members (concatenated, ascending per
@@ -166,7 +170,8 @@ def plan(block_tables, seq_lens, block_size: int, min_group_size: int = 2,
     members = np.zeros(max(cap_m, 1), np.int32)
     ss = np.zeros(R, np.int32)
     rc = _load().oracle_plan(bt.reshape(-1), R, mb, sl, block_size, min_group_size,
-                             min_shared_blocks, ng, a, b, parent, moff, nm, members, ss,
+                             min_shared_blocks, min_saved_blocks, ng, a, b, parent, moff, nm,
+                             members, ss,
                              cap_g, members.shape[0])
     if rc:
         raise RuntimeError(f"oracle_plan failed ({rc})")

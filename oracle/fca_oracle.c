@@ -221,7 +221,7 @@ typedef struct {
     int32_t n_nodes, cap_nodes;
     raw_group *groups;
     int32_t n_groups, cap_groups;
-    int32_t min_group_size, min_shared_blocks;
+    int32_t min_group_size, min_shared_blocks, min_saved_blocks;
 } trie_state;
 
 static int32_t trie_child(trie_state *st, int32_t v, int32_t block)
@@ -254,8 +254,11 @@ static int32_t same_set_child(const trie_state *st, int32_t v)
  * the same member set down to its last node.  Chains with fewer than
  * min_group_size members are not groups, and neither is anything below them.
  * A chain shorter than min_shared_blocks (after absorbing any dropped
- * ancestors, "pending") is dropped: its interval passes to the chains below
- * it, or stays with the members' suffixes if there are none.
+ * ancestors, "pending"), or one whose sharing saves fewer than
+ * min_saved_blocks block reads ((members - 1) x its length in blocks: the
+ * reads of the shared blocks by all but one member), is dropped: its interval
+ * passes to the chains below it, or stays with the members' suffixes if there
+ * are none.
  */
 static int walk_chain(trie_state *st, int32_t start, int32_t parent_group, int32_t pending)
 {
@@ -267,7 +270,8 @@ static int walk_chain(trie_state *st, int32_t start, int32_t parent_group, int32
     int32_t b = nd[end].depth;
     int32_t eff_a = pending >= 0 ? pending : a;
     int32_t next_parent = parent_group, next_pending = -1;
-    if (b - eff_a < st->min_shared_blocks) {
+    if (b - eff_a < st->min_shared_blocks ||
+        (int64_t)(nd[start].count - 1) * (b - eff_a) < (int64_t)st->min_saved_blocks) {
         next_pending = eff_a;
     } else {
         if (st->n_groups == st->cap_groups) return ORACLE_ERR_CAPACITY;
@@ -312,12 +316,13 @@ static int cmp_group_idx(const void *x, const void *y)
  */
 int oracle_plan(const int32_t *block_tables, int32_t R, int32_t max_blocks,
                 const int32_t *seq_lens, int32_t B, int32_t min_group_size,
-                int32_t min_shared_blocks, int32_t *n_groups, int32_t *g_a,
+                int32_t min_shared_blocks, int32_t min_saved_blocks, int32_t *n_groups, int32_t *g_a,
                 int32_t *g_b, int32_t *g_parent, int32_t *g_member_off,
                 int32_t *g_n_members, int32_t *members, int32_t *suffix_start,
                 int32_t cap_groups, int64_t cap_members)
 {
-    if (R <= 0 || max_blocks <= 0 || B <= 0 || min_group_size < 2 || min_shared_blocks < 1)
+    if (R <= 0 || max_blocks <= 0 || B <= 0 || min_group_size < 2 || min_shared_blocks < 1 ||
+        min_saved_blocks < 0)
         return ORACLE_ERR_ARG;
     int64_t total_full = 0;
     for (int32_t r = 0; r < R; ++r) {
@@ -338,6 +343,7 @@ int oracle_plan(const int32_t *block_tables, int32_t R, int32_t max_blocks,
     }
     st.min_group_size = min_group_size;
     st.min_shared_blocks = min_shared_blocks;
+    st.min_saved_blocks = min_saved_blocks;
     st.n_nodes = 1;
     st.nodes[0].block = -1;
     st.nodes[0].depth = 0;

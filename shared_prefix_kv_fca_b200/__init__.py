@@ -51,7 +51,8 @@ class FcaError(RuntimeError):
 
 class fca_plan_opts(ctypes.Structure):
     _fields_ = [("min_group_size", ctypes.c_int32), ("min_shared_blocks", ctypes.c_int32),
-                ("split_tokens", ctypes.c_int32), ("flags", ctypes.c_int32)]
+                ("split_tokens", ctypes.c_int32), ("flags", ctypes.c_int32),
+                ("min_saved_blocks", ctypes.c_int32)]
 
 
 class fca_plan_stats(ctypes.Structure):
@@ -159,15 +160,18 @@ def fca_plan_opts_default() -> fca_plan_opts:
 def fca_plan(block_tables, seq_lens, num_blocks: int, num_q_heads: int, num_kv_heads: int,
              head_dim: int, block_size: int = 16, min_group_size: int = 2,
              min_shared_blocks: int = 1, split_tokens: int = 0, flat: bool = False,
-             stream=None) -> "Plan":
+             stream=None, min_saved_blocks: int = 32) -> "Plan":
     """Group discovery + work lists.  block_tables int32 [R, max_blocks] and
-    seq_lens int32 [R] are CUDA tensors."""
+    seq_lens int32 [R] are CUDA tensors.  min_saved_blocks: groups whose
+    sharing saves fewer block reads ((members - 1) x length in blocks) are
+    folded (0 keeps every shared prefix)."""
     lib = load_library()
     for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens")):
         if not t.is_cuda or str(t.dtype) != "torch.int32" or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
     R, mb = block_tables.shape
-    o = fca_plan_opts(min_group_size, min_shared_blocks, split_tokens, FCA_PLAN_FLAT if flat else 0)
+    o = fca_plan_opts(min_group_size, min_shared_blocks, split_tokens, FCA_PLAN_FLAT if flat else 0,
+                      min_saved_blocks)
     handle = ctypes.c_void_p()
     rc = lib.fca_plan(_ptr(block_tables), mb, _ptr(seq_lens), R, block_size, num_blocks, num_q_heads,
                       num_kv_heads, head_dim, ctypes.byref(o), ctypes.byref(handle),

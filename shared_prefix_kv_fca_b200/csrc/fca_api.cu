@@ -74,6 +74,7 @@ void fca_plan_opts_default(fca_plan_opts* opts) {
     if (!opts) return;
     opts->min_group_size = 2;
     opts->min_shared_blocks = 1;
+    opts->min_saved_blocks = kDefaultMinSavedBlocks;
     opts->split_tokens = 0;
     opts->flags = 0;
 }
@@ -107,7 +108,8 @@ fca_status fca_plan(const int32_t* block_tables, int32_t max_blocks, const int32
     fca_plan_opts o;
     fca_plan_opts_default(&o);
     if (opts) o = *opts;
-    if (o.min_group_size < 2 || o.min_shared_blocks < 1 || o.split_tokens < 0 || o.split_tokens % 64 != 0)
+    if (o.min_group_size < 2 || o.min_shared_blocks < 1 || o.min_saved_blocks < 0 || o.split_tokens < 0 ||
+        o.split_tokens % 64 != 0)
         return FCA_ERR_INVALID_ARG;
     fca_plan_s* P = new (std::nothrow) fca_plan_s();
     if (!P) return FCA_ERR_OOM;

@@ -40,6 +40,15 @@ constexpr size_t kStaticScratchBytes = size_t(64) << 20;
 constexpr double kPrefixGBsPerSM = 18.0;
 constexpr double kSuffixGBsPerSM = 49.0;
 
+// Default of fca_plan_opts.min_saved_blocks: a group is used only if sharing
+// it saves at least this many block reads, (members - 1) x its length in
+// blocks.  A grouped-pass work item costs about as much as streaming 32 blocks
+// of one KV head in the per-request pass (item set-up, query-tile load and
+// epilogue), so smaller groups make the step slower: on 512 pairs of requests
+// sharing 1-16 blocks, keeping every group took 745 us a step against 522 for
+// the flat decode.
+constexpr int32_t kDefaultMinSavedBlocks = 32;
+
 // Shortest chunk the per-request pass splits a request's own tokens into.
 // Longer chunks mean fewer partial rows to write and merge; a sweep of 256,
 // 384 and 512 on the four large workloads favoured 512 (forest 204 -> 195 us

@@ -147,7 +147,7 @@ __global__ void k_check_chain(const int32_t* __restrict__ bt, int32_t MB, int32_
 
 struct RowArgs {
     const int32_t* bt;
-    int32_t MB, R, G, min_group_size, min_shared_blocks, pass;
+    int32_t MB, R, G, min_group_size, min_shared_blocks, min_saved_blocks, pass;
     const int32_t* nfull;
     const int32_t* owner;
     const int32_t* count;
@@ -312,7 +312,10 @@ __global__ void __launch_bounds__(256) k_row_runs(RowArgs args) {
                     const int32_t next_o = __shfl_sync(0xffffffffu, o, src);
                     // close the run [cur_start, kend) with count cur_cnt
                     const int32_t eff_a = pending >= 0 ? pending : cur_start;
-                    if (kend - eff_a < args.min_shared_blocks) {
+                    // too short, or saving too few block reads ((members - 1) x length)
+                    // to pay for its own work items: fold it
+                    if (kend - eff_a < args.min_shared_blocks ||
+                        (int64_t)(cur_cnt - 1) * (kend - eff_a) < (int64_t)args.min_saved_blocks) {
                         pending = eff_a;
                     } else {
                         if (args.pass == 0) {
@@ -904,6 +907,7 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
         ra.G = G;
         ra.min_group_size = opts.min_group_size;
         ra.min_shared_blocks = opts.min_shared_blocks;
+        ra.min_saved_blocks = opts.min_saved_blocks;
         ra.pass = 0;
         ra.nfull = s.nfull;
         ra.owner = s.owner;

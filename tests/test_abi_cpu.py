@@ -54,7 +54,7 @@ def test_host_only_calls(lib):
     assert fca.fca_status_string(0) == "ok"
     assert fca.fca_status_string(2) == "block id out of range"
     o = fca.fca_plan_opts_default()
-    assert (o.min_group_size, o.min_shared_blocks, o.split_tokens, o.flags) == (2, 1, 0, 0)
+    assert (o.min_group_size, o.min_shared_blocks, o.split_tokens, o.flags, o.min_saved_blocks) == (2, 1, 0, 0, 32)
 
 
 def test_argument_checks_return_status_without_a_device(lib):

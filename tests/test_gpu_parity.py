@@ -27,8 +27,11 @@ def _torch():
 
 
 def run(w, flat=False, lse=True, **opts):
-    """Plan + decode through the binding; returns (out f64 [R,Hq,D], lse f64, plan export, stats)."""
+    """Plan + decode through the binding; returns (out f64 [R,Hq,D], lse f64, plan export, stats).
+    Every shared prefix is used (min_saved_blocks 0) unless the caller says
+    otherwise, so that the small random forests exercise the grouped pass."""
     torch = _torch()
+    opts.setdefault("min_saved_blocks", 0)
     import shared_prefix_kv_fca_b200 as fca
     q, k, v, bt, sl = w.torch_inputs("cuda")
     plan = fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, flat=flat, **opts)
@@ -69,12 +72,38 @@ def test_plan_bit_exact_random_forests(seed):
                                                                w.block_size, w.num_blocks)
 
 
-@pytest.mark.parametrize("mgs,msb", [(3, 1), (2, 2), (4, 3), (2, 5)])
-def test_plan_options(mgs, msb):
+@pytest.mark.parametrize("mgs,msb,msv", [(3, 1, 0), (2, 2, 0), (4, 3, 0), (2, 5, 0), (2, 1, 5), (2, 1, 32),
+                                         (3, 2, 12), (2, 1, 1000)])
+def test_plan_options(mgs, msb, msv):
     for seed in range(12):
         w = fca_workloads.random_small(seed, max_requests=24)
-        _, _, exp, _ = run(w, min_group_size=mgs, min_shared_blocks=msb)
-        assert_plan_equal(exp, oracle.plan(w.block_tables, w.seq_lens, w.block_size, mgs, msb))
+        _, _, exp, _ = run(w, min_group_size=mgs, min_shared_blocks=msb, min_saved_blocks=msv)
+        assert_plan_equal(exp, oracle.plan(w.block_tables, w.seq_lens, w.block_size, mgs, msb, msv))
+
+
+def test_default_plan_folds_groups_too_small_to_pay():
+    # the default plan (min_saved_blocks 32) on pairs of requests sharing short
+    # prompts: the groups that save fewer than 32 block reads are folded, the
+    # plan still matches the oracle bit for bit, and decode matches attention
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    w = fca_workloads.make("pairs", prompts=24)
+    q, k, v, bt, sl = w.torch_inputs("cuda")
+    with fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D) as plan:
+        exp = plan.export()
+        out = torch.empty_like(q)
+        lse = torch.empty(w.R, w.Hq, dtype=torch.float32, device="cuda")
+        fca.fca_decode(q, k, v, plan, out, lse, w.scale)
+        assert fca.fca_check_device_status(plan) == 0
+    ref = oracle.plan(w.block_tables, w.seq_lens, 16, min_saved_blocks=32)
+    assert_plan_equal(exp, ref)
+    assert len(ref["a"]) < len(oracle.plan(w.block_tables, w.seq_lens, 16)["a"])
+    pairs = sampled_pairs(w, 64)
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                                          pairs=pairs)
+    sel = (pairs[:, 0], pairs[:, 1])
+    o = out.float().cpu().numpy().astype(np.float64)
+    assert_close(o[sel], lse.cpu().numpy().astype(np.float64)[sel], o_ref, l_ref, "pairs default plan")
 
 
 def inconsistent_workload():

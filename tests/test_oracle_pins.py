@@ -293,6 +293,70 @@ def test_plan_min_shared_blocks_folds_short_groups():
     assert list(p["suffix_start"]) == [6, 6, 0, 0]
 
 
+def test_plan_min_saved_blocks_hand_example():
+    # three groups: r0,r1 share 3 blocks (saves 1 x 3 block reads), r2..r5
+    # share 10 (3 x 10 = 30), r6..r9 share 12 (3 x 12 = 36)
+    B = 16
+    rows, lens = [], []
+    nxt = 1000
+    for members, shared, base in ((2, 3, 100), (4, 10, 200), (4, 12, 300)):
+        for _ in range(members):
+            rows.append([base + j for j in range(shared)] + [nxt])
+            lens.append((shared + 1) * B)
+            nxt += 1
+    mb = max(len(x) for x in rows)
+    bt = np.array([x + [0] * (mb - len(x)) for x in rows], np.int32)
+    sl = np.array(lens, np.int32)
+    for T, kept in ((0, [2, 4, 4]), (3, [2, 4, 4]), (4, [4, 4]), (30, [4, 4]), (31, [4]), (36, [4]), (37, [])):
+        p = oracle.plan(bt, sl, B, min_saved_blocks=T)
+        assert list(p["n_members"]) == kept, (T, p["n_members"])
+        saved = [(int(n) - 1) * (int(b) - int(a)) for n, a, b in zip(p["n_members"], p["a"], p["b"])]
+        assert all(x >= T for x in saved)
+        # members of a folded group read their whole table in their own pass
+        ss = np.zeros(len(rows), np.int32)
+        for g in range(len(p["a"])):
+            for m in p["members"][p["member_off"][g]:p["member_off"][g] + p["n_members"][g]]:
+                ss[m] = p["b"][g]
+        assert list(p["suffix_start"]) == list(ss)
+
+
+@pytest.mark.parametrize("T", [2, 5, 12, 40])
+def test_plan_min_saved_blocks_properties(T):
+    """Against the unfolded forest (pinned by the all-pairs LCP test): kept
+    groups are unfolded groups whose interval starts at the end of their
+    nearest kept ancestor; a group is kept exactly when (members - 1) x that
+    interval's length reaches T; suffix starts follow the kept groups."""
+    for seed in range(20):
+        w = fca_workloads.random_small(seed, max_requests=16)
+        full = oracle.plan(w.block_tables, w.seq_lens, w.block_size)
+        fold = oracle.plan(w.block_tables, w.seq_lens, w.block_size, min_saved_blocks=T)
+        def sets(p):
+            return [frozenset(int(x) for x in p["members"][p["member_off"][g]:p["member_off"][g] + p["n_members"][g]])
+                    for g in range(len(p["a"]))]
+        fs, ks = sets(full), sets(fold)
+        kept_b = {(S, int(b)): int(a) for S, a, b in zip(ks, fold["a"], fold["b"])}
+        # walk the unfolded forest root first (canonical order lists parents first)
+        kept_end = {}
+        for g in range(len(fs)):
+            par = int(full["parent"][g])
+            start = 0
+            q = par
+            while q >= 0 and q not in kept_end:
+                q = int(full["parent"][q])
+            if q >= 0:
+                start = kept_end[q]
+            length = int(full["b"][g]) - start
+            keep = (len(fs[g]) - 1) * length >= T and length >= 1
+            assert ((fs[g], int(full["b"][g])) in kept_b) == keep, (seed, g)
+            if keep:
+                assert kept_b[(fs[g], int(full["b"][g]))] == start
+                kept_end[g] = int(full["b"][g])
+        assert len(ks) == len(kept_end)
+        for r in range(w.R):
+            deepest = max([int(b) for S, b in zip(ks, fold["b"]) if r in S], default=0)
+            assert fold["suffix_start"][r] == deepest
+
+
 def test_plan_partial_blocks_and_identical_tables():
     B = 16
     bt = np.array([[3, 4, 5], [3, 4, 5], [3, 4, 6], [3, 9, 9]], np.int32)
