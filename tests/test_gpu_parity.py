@@ -384,3 +384,82 @@ def test_error_paths_return_status():
         out = torch.empty_like(q)
         fca.fca_decode(q, k, v, plan, out)
         assert fca.fca_check_device_status(plan) == 0
+
+
+# --------------------------------------------------------------- limits and degenerate shapes
+
+def test_plan_and_decode_at_the_request_limit():
+    # 16384 requests (the planner's limit): 1024 prompts of 2-3 blocks x 16
+    # samples with 1..20 own tokens; head_dim 64, one KV head
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    rng = np.random.default_rng(77)
+    reqs = []
+    for p in range(1024):
+        plen = int(rng.integers(32, 49))
+        for _ in range(16):
+            reqs.append([(f"p{p}", plen), (None, int(rng.integers(1, 21)))])
+    w = fca_workloads.fill("limit", reqs, Hq=4, Hkv=1, D=64, seed=77, rng=rng)
+    assert w.R == 16384
+    o, l, exp, st = run(w)
+    assert_plan_equal(exp, oracle.plan(w.block_tables, w.seq_lens, 16))
+    assert st["num_groups"] == 1024
+    pairs = sampled_pairs(w, 96, 3)
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                                          pairs=pairs)
+    sel = (pairs[:, 0], pairs[:, 1])
+    assert_close(o[sel], l[sel], o_ref, l_ref, "request limit")
+    # one request more is refused, without touching the device state
+    bt = torch.from_numpy(np.concatenate([w.block_tables, w.block_tables[:1]])).cuda()
+    sl = torch.from_numpy(np.concatenate([w.seq_lens, w.seq_lens[:1]])).cuda()
+    with pytest.raises(fca.FcaError) as e:
+        fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D)
+    assert e.value.status == 3
+
+
+def test_fallback_planner_limit():
+    # tables whose block ids do not identify prefixes take the all-pairs
+    # planner, which handles up to 4096 requests; past that the plan is refused
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    base = inconsistent_workload()
+    for R, ok in ((4096, True), (4100, False)):
+        reps = (R + base.R - 1) // base.R
+        bt = np.tile(base.block_tables, (reps, 1))[:R]
+        sl = np.tile(base.seq_lens, reps)[:R]
+        if ok:
+            w = fca_workloads.Workload("fallback_limit", fca_workloads.normal_bf16((R, base.Hq, base.D), 8, 0),
+                                       base.k_cache, base.v_cache, bt, sl, base.Hq, base.Hkv, base.D, 16, 8)
+            o, l, exp, _ = run(w)
+            assert_plan_equal(exp, oracle.plan(bt, sl, 16))
+            pairs = sampled_pairs(w, 48, 5)
+            o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, bt, sl, w.scale, pairs=pairs)
+            sel = (pairs[:, 0], pairs[:, 1])
+            assert_close(o[sel], l[sel], o_ref, l_ref, "fallback at its limit")
+        else:
+            with pytest.raises(fca.FcaError) as e:
+                fca.fca_plan(torch.from_numpy(bt).cuda(), torch.from_numpy(sl).cuda(), base.num_blocks, base.Hq,
+                             base.Hkv, base.D)
+            assert e.value.status == 3
+
+
+@pytest.mark.parametrize("case", ["single_request", "identical_full_tables", "one_token", "full_table"])
+def test_degenerate_batches(case):
+    rng = np.random.default_rng(11)
+    if case == "single_request":
+        reqs = [[(None, 77)]]
+    elif case == "identical_full_tables":
+        # every token of every request is shared: no own tokens at all
+        reqs = [[("p", 96)] for _ in range(6)]
+    elif case == "one_token":
+        reqs = [[(None, 1)] for _ in range(5)] + [[("p", 16), (None, 1)] for _ in range(3)]
+    else:
+        # sequences that end exactly on a block boundary, one at max_blocks * 16
+        reqs = [[("p", 64), (None, 64)] for _ in range(4)] + [[("p", 64), (None, 128)]]
+    w = fca_workloads.fill(case, reqs, Hq=8, Hkv=2, D=128, seed=11, rng=rng, poison_padding=True)
+    o, l, exp, _ = run(w)
+    assert_plan_equal(exp, oracle.plan(w.block_tables, w.seq_lens, 16))
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(o, l, o_ref, l_ref, case)
+    if case == "identical_full_tables":
+        assert list(exp["suffix_start"]) == [6] * 6
