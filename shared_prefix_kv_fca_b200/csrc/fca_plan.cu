@@ -10,7 +10,10 @@
 // The forest is the trie of the requests' full-block id sequences: a node is
 // a prefix, its member set is the requests whose tables start with it, and a
 // group is a maximal run of depths over which the member set does not change
-// (and has at least min_group_size members).
+// (and has at least min_group_size members).  A group shorter than
+// min_shared_blocks, or one whose sharing saves fewer than min_saved_blocks
+// block reads ((members - 1) x length), is folded: its interval passes to the
+// groups below it, or to its members' own passes.
 //
 // Fast path (every table produced by a prefix-caching allocator).  A trie node
 // at depth k + 1 is identified by the physical block at logical index k,
@@ -512,8 +515,9 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
 
     // Chunk targets.  The grouped pass runs one CTA per SM, so aim at about
     // three items per SM; the per-request pass runs one item per warp, eight
-    // warps per SM, so aim at about four items per warp.  Each group / request
-    // then splits its tokens evenly into chunks of at most the target.
+    // warps per SM, so aim at about four items per warp, with chunks of at
+    // least kMinOwnChunk tokens.  Each group / request then splits its tokens
+    // evenly into chunks of at most the target.
     const int32_t tile_rows = kPrefixTileRows;
     int64_t wp = 0, ws = 0;
     for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
