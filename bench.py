@@ -2,7 +2,7 @@
 """Benchmark of one FCA decode step (one layer) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fca|reference]
-                    [--config llama8b|longctx|forest|mixed|tiny]
+                    [--config llama8b|longctx|forest|mixed|pairs|tiny] [--layers L]
 
 A step is one pass of the whole hot path -- grouped prefix pass, per-request
 pass, log-sum-exp merge -- over the configuration's synthetic batch, with the
@@ -106,7 +106,6 @@ class ClockSampler:
     def stop(self):
         if self.proc is None:
             return None
-        time.sleep(0.25)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -131,10 +130,11 @@ class ClockSampler:
             for name, val in zip(names, r[5:9]):
                 if val.lower() == "active":
                     reasons.add(name)
-        loaded = [s for s, p in zip(sm, pw) if p >= 200.0] or sm
+        busy = [s for s, p in zip(sm, pw) if p >= 200.0]
+        loaded = busy or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(busy),
                 "power_w_max": max(pw) if pw else None}
 
 
@@ -361,11 +361,20 @@ def fca_arm(args):
     sampler = ClockSampler(gpu_id_for(local)) if rank == 0 else None
     barrier()
     torch.cuda.synchronize(dev)
+    def keep_busy(seconds):
+        """Untimed steps of the same workload around the timed region, so that
+        the clock samples (every 200 ms) see the GPU under this load."""
+        t_end = time.perf_counter() + seconds
+        while time.perf_counter() < t_end:
+            run_steps(plan, 8, False)
+
     if sampler:
         sampler.start()
-        time.sleep(0.3)
+        keep_busy(0.6)
     step_ms_rank = run_steps(plan, args.steps, True)
     torch.cuda.synchronize(dev)
+    if sampler:
+        keep_busy(0.6)
     clocks = sampler.stop() if sampler else None
     barrier()
     assert fca.fca_check_device_status(plan, stream) == 0

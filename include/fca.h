@@ -27,6 +27,10 @@
  *   - Pointers marked DEVICE are CUDA device pointers on the current device;
  *     HOST pointers are ordinary host memory.  The caller owns every buffer it
  *     passes in; the library owns only what a plan handle holds.
+ *   - A plan belongs to the device that was current when it was built.  Calls
+ *     that take a plan run on that device (made current for the call, the
+ *     caller's current device restored on return); their buffers and stream
+ *     must belong to it.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls that
  *     take a stream are asynchronous on it unless stated otherwise.
  *   - Functions return fca_status; nothing throws, traps or aborts across the

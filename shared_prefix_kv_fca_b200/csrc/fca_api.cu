@@ -64,6 +64,20 @@ bool make_cache_map(CUtensorMap* map, const void* base, int32_t num_blocks, int3
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Makes a plan's device current for one call and restores the caller's
+// device afterwards (a no-op when it is current already).
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        int cur = 0;
+        if (cudaGetDevice(&cur) == cudaSuccess && cur != dev && cudaSetDevice(dev) == cudaSuccess) prev = cur;
+        (void)cudaGetLastError();
+    }
+    ~DeviceGuard() {
+        if (prev >= 0) cudaSetDevice(prev);
+    }
+};
+
 }  // namespace fca
 
 using namespace fca;
@@ -81,6 +95,7 @@ void fca_plan_opts_default(fca_plan_opts* opts) {
 
 fca_status fca_plan_destroy(fca_plan_t plan) {
     if (!plan) return FCA_OK;
+    DeviceGuard dg(plan->device);
     // the plan's memory goes back to the library's pool once nothing that may
     // read it is still running
     cudaDeviceSynchronize();
@@ -150,6 +165,7 @@ static fca_status decode_impl(const void* q, const void* k_cache, const void* v_
                               float* lse, float scale, void* stream) {
     if (!plan || !q || !k_cache || !v_cache || !out) return FCA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !(scale < INFINITY)) return FCA_ERR_INVALID_ARG;
+    DeviceGuard dg(plan->device);
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return FCA_ERR_INVALID_ARG;
@@ -199,6 +215,7 @@ static fca_status pass_impl(int pass, const void* q, const void* k_cache, const 
                             float scale, void* stream) {
     if (!plan || !q || !k_cache || !v_cache) return FCA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !(scale < INFINITY)) return FCA_ERR_INVALID_ARG;
+    DeviceGuard dg(plan->device);
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return FCA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     CUtensorMap tk, tv;
@@ -226,6 +243,7 @@ fca_status fca_suffix_pass(const void* q, const void* k_cache, const void* v_cac
 fca_status fca_merge_pass(fca_plan_t plan, void* out, float* lse, void* stream) {
     if (!plan || !out || !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return FCA_ERR_INVALID_ARG;
+    DeviceGuard dg(plan->device);
     return note_cuda(launch_merge(plan, out, lse, static_cast<cudaStream_t>(stream))) == cudaSuccess
                ? FCA_OK
                : FCA_ERR_CUDA;
@@ -271,6 +289,7 @@ fca_status fca_plan_member_count(fca_plan_t plan, int64_t* count) {
 fca_status fca_plan_export(fca_plan_t plan, int32_t* a, int32_t* b, int32_t* parent, int32_t* member_off,
                            int32_t* n_members, int32_t* members, int32_t* suffix_start) {
     if (!plan) return FCA_ERR_INVALID_ARG;
+    DeviceGuard dg(plan->device);
     if (cudaDeviceSynchronize() != cudaSuccess) {
         (void)cudaGetLastError();
         return FCA_ERR_CUDA;
@@ -299,6 +318,7 @@ fca_status fca_plan_export(fca_plan_t plan, int32_t* a, int32_t* b, int32_t* par
 
 fca_status fca_check_device_status(fca_plan_t plan, void* stream, int32_t* code) {
     if (!plan) return FCA_ERR_INVALID_ARG;
+    DeviceGuard dg(plan->device);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t v = 0;
     if (cudaStreamSynchronize(s) != cudaSuccess ||
