@@ -130,6 +130,8 @@ struct fca_plan_s {
     int32_t* g_nch = nullptr;        // split chunks of the group's token range
     int32_t* g_chunk = nullptr;      // tokens per chunk (last one may be shorter)
     int32_t* g_part = nullptr;       // partial row of (group, head 0, chunk 0, row 0)
+    int32_t* g_wa = nullptr;         // first block of the group's grouped-pass items (its a, or
+                                     // its parent's when the parent is folded into its children)
     int32_t* members = nullptr;      // [n_member_entries]
     int32_t* suffix_start = nullptr; // [R] blocks
     int32_t* chain_off = nullptr;    // [R + 1] into chain_g / chain_pos

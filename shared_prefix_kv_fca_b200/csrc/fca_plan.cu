@@ -43,6 +43,12 @@
 
 #include "fca_internal.h"
 
+// A group's grouped-pass work up to this many times the chunk target stays one
+// item (sweep of 1.0 / 1.5 / 2.0 on four workloads: 1.5 and 2.0 took the
+// llama8b step from 141 to 139 us and the forest's from 201 to 193 once its
+// root is folded into its prompts' items; 1.0 is the plain ceiling).
+constexpr double kWholeItem = 1.5;
+
 namespace fca {
 namespace {
 
@@ -66,6 +72,7 @@ struct PlanScratch {
     uint64_t* keys;        // [R] canonical (a << 32 | owner)
     int32_t* g_item_off;   // [R + 1]
     int32_t* s_item_off;   // [R + 1]
+    int32_t* gwork;        // [4 R] per group: children's members, tiles, count, non-leaf count
     PlanHeader* hdr;       // [1]
 };
 
@@ -456,6 +463,7 @@ struct FinalizeArgs {
     int32_t* chain_off;  // [R + 1]
     int32_t* g_chunk;
     int32_t* s_chunk;
+    int32_t* g_wa;       // first block of each group's grouped-pass items
     int32_t* bin_cursor; // [kBins] first item slot of each length bin, longest first
     int32_t num_sms;
 };
@@ -512,17 +520,57 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
         }
         A.g_parent[i] = par;
     }
+    __syncthreads();
+
+    // A group whose members all belong to its child groups, whose children are
+    // leaves, and whose children need no more 128-row query tiles than it
+    // does, has no work items of its own: each child's items start at the
+    // parent's first block instead (a member's tables agree on the parent's
+    // interval and the child's), so the parent's blocks are streamed the same
+    // number of times, by fewer and longer items, with one partial row per
+    // member fewer to write and merge.  (The forest of a system prompt over
+    // several prompts: the root's tiles are the prompts' tiles.)
+    const int32_t tile_rows = kPrefixTileRows;
+    auto tiles_of = [&](int32_t i) { return (A.g_nm[i] * G + tile_rows - 1) / tile_rows; };
+    int32_t* c_nm = A.s.gwork;
+    int32_t* c_tiles = c_nm + R;
+    int32_t* c_count = c_tiles + R;
+    int32_t* c_inner = c_count + R;   // children that have children; -1 marks a folded-in parent
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x) c_nm[i] = c_tiles[i] = c_count[i] = c_inner[i] = 0;
+    __syncthreads();
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const int32_t par = A.g_parent[i];
+        if (par >= 0) {
+            atomicAdd(&c_nm[par], A.g_nm[i]);
+            atomicAdd(&c_tiles[par], tiles_of(i));
+            atomicAdd(&c_count[par], 1);
+        }
+    }
+    __syncthreads();
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const int32_t par = A.g_parent[i];
+        if (par >= 0 && c_count[i] > 0) atomicAdd(&c_inner[par], 1);
+    }
+    __syncthreads();
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x)
+        if (c_count[i] > 0 && c_inner[i] == 0 && c_nm[i] == A.g_nm[i] && c_tiles[i] <= tiles_of(i)) c_inner[i] = -1;
+    __syncthreads();
+    auto folded_in = [&](int32_t i) { return c_inner[i] < 0; };
+    for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const int32_t par = A.g_parent[i];
+        A.g_wa[i] = (par >= 0 && folded_in(par)) ? A.g_a[par] : A.g_a[i];
+    }
+    __syncthreads();
 
     // Chunk targets.  The grouped pass runs one CTA per SM, so aim at about
     // three items per SM; the per-request pass runs one item per warp, eight
     // warps per SM, so aim at about four items per warp, with chunks of at
     // least kMinOwnChunk tokens.  Each group / request then splits its tokens
     // evenly into chunks of at most the target.
-    const int32_t tile_rows = kPrefixTileRows;
     int64_t wp = 0, ws = 0;
     for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
-        const int64_t tok = (int64_t)(A.g_b[i] - A.g_a[i]) * kBlockSize;
-        wp += tok * ((A.g_nm[i] * G + tile_rows - 1) / tile_rows);
+        const int64_t tok = folded_in(i) ? 0 : (int64_t)(A.g_b[i] - A.g_wa[i]) * kBlockSize;
+        wp += tok * tiles_of(i);
     }
     for (int32_t r = threadIdx.x; r < R; r += blockDim.x)
         ws += A.seq_lens[r] - (int64_t)A.suffix_start[r] * kBlockSize;
@@ -551,9 +599,18 @@ __global__ void __launch_bounds__(1024) k_finalize(FinalizeArgs A) {
                                                    A.g_moff, red);
     for (int32_t i = threadIdx.x; i < n; i += blockDim.x) {
         // chunks are whole stages of the grouped pass; their count follows
-        // from the rounded size, so that every chunk holds tokens
-        const int32_t tok = (A.g_b[i] - A.g_a[i]) * kBlockSize;
-        const int32_t want = (tok + split_p - 1) / split_p;
+        // from the rounded size, so that every chunk holds tokens (a group
+        // folded into its children has none)
+        if (folded_in(i)) {
+            A.g_chunk[i] = 0;
+            A.g_nch[i] = 0;
+            continue;
+        }
+        const int32_t tok = (A.g_b[i] - A.g_wa[i]) * kBlockSize;
+        // a group's work up to kWholeItem x the target stays one chunk: an item
+        // costs a fixed set-up and epilogue on top of its stages, so one long
+        // item beats two short ones unless the balance across CTAs needs them
+        const int32_t want = tok <= (int32_t)(kWholeItem * split_p) ? 1 : (tok + split_p - 1) / split_p;
         const int32_t chunk = ((tok + want - 1) / want + kStageTokens - 1) / kStageTokens * kStageTokens;
         A.g_chunk[i] = chunk;
         A.g_nch[i] = (tok + chunk - 1) / chunk;
@@ -667,8 +724,10 @@ __global__ void __launch_bounds__(256) k_sort_members(const PlanHeader* hdr, con
 
 // ------------------------------------------------------------ work lists
 
-// One CTA per group: items (q-tile, chunk, head), heads innermost.
-__global__ void k_fill_prefix_items(const PlanHeader* hdr, const int32_t* g_a, const int32_t* g_b,
+// One CTA per group: items (q-tile, chunk, head), heads innermost, over the
+// group's work interval [g_wa, g_b) (g_wa is the parent's first block when the
+// parent is folded into its children).
+__global__ void k_fill_prefix_items(const PlanHeader* hdr, const int32_t* g_wa, const int32_t* g_b,
                                     const int32_t* g_nm, const int32_t* g_moff, const int32_t* g_nch,
                                     const int32_t* g_chunk, const int32_t* g_part, const int32_t* item_off,
                                     const int32_t* members, int32_t G, int32_t Hkv, PrefixItem* items) {
@@ -676,7 +735,7 @@ __global__ void k_fill_prefix_items(const PlanHeader* hdr, const int32_t* g_a, c
     for (int32_t g = blockIdx.x; g < ng; g += gridDim.x) {
         const int32_t rows = g_nm[g] * G, tiles = (rows + kPrefixTileRows - 1) / kPrefixTileRows;
         const int32_t nch = g_nch[g], per_head = tiles * nch, split = g_chunk[g];
-        const int32_t t0 = g_a[g] * kBlockSize, t1 = g_b[g] * kBlockSize;
+        const int32_t t0 = g_wa[g] * kBlockSize, t1 = g_b[g] * kBlockSize;
         // heads innermost: the KV heads of one token are neighbours in the cache
         // (one DRAM row holds all of them), so their items should run together
         for (int32_t i = threadIdx.x; i < Hkv * per_head; i += blockDim.x) {
@@ -844,6 +903,7 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     ta.add(&s.keys, R);
     ta.add(&s.g_item_off, R + 1);
     ta.add(&s.s_item_off, R + 1);
+    ta.add(&s.gwork, (size_t)4 * R);
     ta.add(&bin_cursor, kBins);
     TempArena tmp(stream);
     if (ta.commit(stream, &tmp.base) != cudaSuccess) {
@@ -872,6 +932,7 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     pa.add(&P->s_part, R + 1);
     pa.add(&P->g_chunk, R);
     pa.add(&P->s_chunk, R);
+    pa.add(&P->g_wa, R);
     pa.add(&P->chain_off, R + 1);
     {
         void* base = nullptr;
@@ -946,6 +1007,7 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     fa.chain_off = P->chain_off;
     fa.g_chunk = P->g_chunk;
     fa.s_chunk = P->s_chunk;
+    fa.g_wa = P->g_wa;
     fa.bin_cursor = bin_cursor;
     {
         int dev = 0;
@@ -1002,7 +1064,7 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
         k_sort_members<<<std::min(H.n_groups, 148 * 4), 256, mem_smem, stream>>>(
             s.hdr, P->g_moff, P->g_nm, P->members, P->chain_off, P->chain_g, P->chain_pos);
         k_fill_prefix_items<<<std::min(H.n_groups, 148 * 4), 256, 0, stream>>>(
-            s.hdr, P->g_a, P->g_b, P->g_nm, P->g_moff, P->g_nch, P->g_chunk, P->g_part, s.g_item_off, P->members,
+            s.hdr, P->g_wa, P->g_b, P->g_nm, P->g_moff, P->g_nch, P->g_chunk, P->g_part, s.g_item_off, P->members,
             G, Hkv, P->prefix_items);
         FCA_CK(cudaGetLastError());
     }

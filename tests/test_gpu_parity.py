@@ -463,3 +463,31 @@ def test_degenerate_batches(case):
     assert_close(o, l, o_ref, l_ref, case)
     if case == "identical_full_tables":
         assert list(exp["suffix_start"]) == [6] * 6
+
+
+@pytest.mark.parametrize("cover", [True, False])
+def test_parent_folded_into_child_items(cover):
+    # 16 query heads per KV head: a 16-member system-prompt group is 256 rows
+    # (two tiles) and each of its two 8-member prompt groups one tile, so the
+    # root's blocks can be streamed inside its children's items; with one
+    # member that has no prompt of its own the root keeps its own items
+    rng = np.random.default_rng(41)
+    reqs = []
+    for p in range(2):
+        for _ in range(8):
+            reqs.append([("sys", 64), (f"p{p}", 80), (None, int(rng.integers(1, 40)))])
+    if not cover:
+        reqs.append([("sys", 64), (None, 30)])
+    w = fca_workloads.fill("fold_in", reqs, Hq=16, Hkv=1, D=128, seed=41, rng=rng, poison_padding=True)
+    o, l, exp, st = run(w)
+    ref = oracle.plan(w.block_tables, w.seq_lens, 16)
+    assert_plan_equal(exp, ref)
+    assert len(ref["a"]) == 3
+    # folded: only the two prompt groups have items (one tile each, one chunk);
+    # kept: the root adds its own tiles (17 members x 16 rows = three tiles)
+    if cover:
+        assert st["prefix_items"] == 2
+    else:
+        assert st["prefix_items"] >= 5
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(o, l, o_ref, l_ref, f"fold-in cover={cover}")
