@@ -36,7 +36,11 @@
  *    the same physical block id at the same logical index ("How PagedAttention
  *    Works" step 4: requests with the same prompt reference the same physical
  *    blocks; a block that will diverge is copied first, so only full blocks are
- *    shared).
+ *    shared).  Two options fold groups away (their interval passes to the
+ *    groups below them, or to their members' own passes): min_shared_blocks
+ *    (a group shorter than that) and min_saved_blocks (a group whose sharing
+ *    saves fewer block reads, (members - 1) x length; the reading of FCA's
+ *    automatic activation, "How It Works").
  *
  * All floating point is fp64 on the exact values of the bf16 inputs.
  */
