@@ -58,6 +58,8 @@ def parse():
                     help="shrink the configuration to this many prompts (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true",
+                    help="no clock sampling and no untimed steps around the timed region (profiling runs)")
     ap.add_argument("--no-flat", action="store_true")
     ap.add_argument("--layers", type=int, default=1,
                     help="also time a multi-layer step: one plan, then this many layers' decodes")
@@ -358,23 +360,27 @@ def fca_arm(args):
 
     # ---- FCA, timed region
     run_steps(plan, args.warmup, False)
-    sampler = ClockSampler(gpu_id_for(local)) if rank == 0 else None
+    sampler = ClockSampler(gpu_id_for(local)) if rank == 0 and not args.no_clocks else None
     barrier()
     torch.cuda.synchronize(dev)
     def keep_busy(seconds):
         """Untimed steps of the same workload around the timed region, so that
         the clock samples (every 200 ms) see the GPU under this load."""
+        if args.no_clocks:
+            return
         t_end = time.perf_counter() + seconds
         while time.perf_counter() < t_end:
             run_steps(plan, 8, False)
 
     if sampler:
         sampler.start()
-        keep_busy(0.6)
+    keep_busy(0.6)   # every rank, so that the ranks' timed regions run at the same time
+    barrier()
+    torch.cuda.synchronize(dev)
     step_ms_rank = run_steps(plan, args.steps, True)
     torch.cuda.synchronize(dev)
-    if sampler:
-        keep_busy(0.6)
+    barrier()
+    keep_busy(0.6)
     clocks = sampler.stop() if sampler else None
     barrier()
     assert fca.fca_check_device_status(plan, stream) == 0
