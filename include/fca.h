@@ -120,6 +120,33 @@ fca_status fca_plan(const int32_t *block_tables, int32_t max_blocks, const int32
                     const fca_plan_opts *opts, fca_plan_t *out_plan, void *stream);
 
 /*
+ * fca_plan_update -- the plan for the next decode step of the same batch,
+ * without group discovery.  Between decode steps a request's table only grows
+ * (new blocks for its new tokens, written by that request alone), so the
+ * forest of shared prefixes stays what it was; only the requests' own ranges
+ * and the work lists of the per-request pass change.  Groups are not
+ * rediscovered: blocks shared for the first time after the plan was built are
+ * read by each request's own pass (still exact, just not deduplicated) until
+ * a fresh fca_plan.
+ *
+ *   block_tables, max_blocks, seq_lens, num_requests  as for fca_plan; the
+ *                 same num_requests and max_blocks as the plan (else
+ *                 FCA_ERR_INVALID_ARG).  Each request's first suffix_start
+ *                 blocks (the ones its groups read) must be unchanged and its
+ *                 seq_len must still cover them.
+ *
+ * Synchronises `stream` once (the new sizes), like fca_plan; may take more
+ * memory from the plan pool if the own work outgrew the plan.  Errors:
+ * FCA_ERR_INVALID_ARG (a shared entry changed, a length no longer covers the
+ * shared blocks or is out of range), FCA_ERR_BAD_BLOCK_ID, FCA_ERR_CUDA,
+ * FCA_ERR_OOM; on an error the plan is left as it was.  Not part of the
+ * method's steps: it is "Core Mechanism" step 1 carried over from one decode
+ * step to the next.
+ */
+fca_status fca_plan_update(fca_plan_t plan, const int32_t *block_tables, int32_t max_blocks,
+                           const int32_t *seq_lens, int32_t num_requests, void *stream);
+
+/*
  * fca_decode -- steps 2-4 of "Core Mechanism": the grouped prefix pass, the
  * per-request suffix pass and the log-sum-exp merge, for one layer.
  *

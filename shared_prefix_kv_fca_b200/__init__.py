@@ -104,6 +104,8 @@ def load_library():
     lib.fca_plan_export.restype = ctypes.c_int
     lib.fca_plan_member_count.argtypes = [vp, ctypes.POINTER(ctypes.c_int64)]
     lib.fca_plan_member_count.restype = ctypes.c_int
+    lib.fca_plan_update.argtypes = [vp, vp, i32, vp, i32, vp]
+    lib.fca_plan_update.restype = ctypes.c_int
     lib.fca_plan_destroy.argtypes = [vp]
     lib.fca_plan_destroy.restype = ctypes.c_int
     lib.fca_check_device_status.argtypes = [vp, vp, i32p]
@@ -316,6 +318,16 @@ class Plan:
 
     def stats(self) -> dict:
         return fca_plan_get_stats(self)
+
+    def update(self, block_tables, seq_lens, stream=None) -> None:
+        """Next decode step of the same batch (fca_plan_update): new lengths
+        and grown tables over this plan's forest."""
+        for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens")):
+            if not t.is_cuda or str(t.dtype) != "torch.int32" or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+        R, mb = block_tables.shape
+        _check(load_library().fca_plan_update(self.handle, _ptr(block_tables), mb, _ptr(seq_lens), R,
+                                              _stream_handle(stream)), "fca_plan_update")
 
     def export(self) -> dict:
         return fca_plan_export(self)

@@ -11,6 +11,7 @@
 
 namespace fca {
 fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cudaStream_t stream, fca_plan_s* P);
+fca_status plan_update(const int32_t* block_tables, const int32_t* seq_lens, cudaStream_t stream, fca_plan_s* P);
 cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
                           float scale, int max_ctas, cudaStream_t stream);
 cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -146,6 +147,16 @@ fca_status fca_plan(const int32_t* block_tables, int32_t max_blocks, const int32
     }
     *out_plan = P;
     return FCA_OK;
+}
+
+fca_status fca_plan_update(fca_plan_t plan, const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens,
+                           int32_t num_requests, void* stream) {
+    if (!plan || !block_tables || !seq_lens) return FCA_ERR_INVALID_ARG;
+    if (max_blocks != plan->max_blocks || num_requests != plan->R) return FCA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return FCA_ERR_INVALID_ARG;
+    DeviceGuard dg(plan->device);
+    return plan_update(block_tables, seq_lens, static_cast<cudaStream_t>(stream), plan);
 }
 
 // SMs given to the grouped pass when it runs beside the per-request pass:

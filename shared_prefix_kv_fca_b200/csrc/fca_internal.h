@@ -60,6 +60,7 @@ constexpr int32_t kPlanBadSeqLen = 1;
 constexpr int32_t kPlanBadBlockId = 2;
 constexpr int32_t kPlanInconsistent = 4;   // block ids do not identify prefixes
 constexpr int32_t kPlanTooManyGroups = 8;
+constexpr int32_t kPlanUpdateMismatch = 16;   // fca_plan_update: a shared entry or length no longer fits
 
 // One tile of the grouped prefix pass: rows [row0, row0 + nrows) of a
 // group's stacked queries (member i / G, query head head * G + i % G; the
@@ -117,6 +118,8 @@ struct fca_plan_s {
     bool flat = false;
     fca::PlanHeader hdr{};
     size_t workspace_bytes = 0;
+    int64_t cap_suffix_items = 0;    // capacity of suffix_items (fca_plan_update may need more)
+    int64_t cap_partials = 0;        // capacity of part_o / part_lse, in rows
 
     // copies of the inputs
     int32_t* bt = nullptr;           // [R][max_blocks]

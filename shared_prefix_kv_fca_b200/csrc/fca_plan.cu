@@ -779,6 +779,97 @@ __global__ void k_fill_suffix_items(int32_t R, const int32_t* seq_lens, const in
     }
 }
 
+// ------------------------------------------------------------ plan update
+
+// Thread (r, j): the entries of request r's table that its groups read (its
+// first suffix_start[r] blocks) must be the plan's, and its length must still
+// cover them.
+__global__ void k_check_shared(const int32_t* __restrict__ bt_new, const int32_t* __restrict__ sl_new,
+                               const int32_t* __restrict__ bt_old, const int32_t* __restrict__ suffix_start,
+                               int32_t R, int32_t MB, PlanHeader* hdr) {
+    const int64_t total = (int64_t)R * MB;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t r = (int32_t)(i / MB), j = (int32_t)(i % MB);
+        const int32_t ss = suffix_start[r];
+        if (j == 0 && (int64_t)sl_new[r] < (int64_t)ss * kBlockSize) atomicOr(&hdr->status, kPlanUpdateMismatch);
+        if (j < ss && bt_new[i] != bt_old[i]) atomicOr(&hdr->status, kPlanUpdateMismatch);
+    }
+}
+
+struct UpdateOwnArgs {
+    int32_t R, Hkv, G, split_opt, num_sms;
+    int64_t n_ppart;               // partial rows of the grouped pass (unchanged)
+    const int32_t* seq_lens;       // the new lengths
+    const int32_t* suffix_start;   // the plan's
+    int32_t* nch;                  // [R] own chunks
+    int32_t* chunk;                // [R] tokens per own chunk
+    int32_t* part;                 // [R + 1] first partial row of (r, head 0, chunk 0)
+    int32_t* s_item_off;           // [R + 1]
+    int32_t* bin_cursor;           // [kBins]
+    PlanHeader* hdr;
+};
+
+// The own-pass half of k_finalize for new lengths over an unchanged forest:
+// chunk targets, chunks, length bins, item offsets, partial rows and sizes.
+// One CTA of 1024 threads; shared memory: 64 + 1024 int64 of reduction space
+// and kBins int32.
+__global__ void __launch_bounds__(1024) k_update_own(UpdateOwnArgs A) {
+    extern __shared__ int64_t sm_upd[];
+    int64_t* red = sm_upd;
+    int32_t* bins = reinterpret_cast<int32_t*>(red + 64 + 1024);
+    PlanHeader* hdr = A.hdr;
+    if (hdr->status) return;   // the update is refused; nothing to compute
+    const int32_t R = A.R, G = A.G;
+    int64_t ws = 0, ftok = 0;
+    for (int32_t r = threadIdx.x; r < R; r += blockDim.x) {
+        ws += A.seq_lens[r] - (int64_t)A.suffix_start[r] * kBlockSize;
+        ftok += A.seq_lens[r];
+    }
+    ws = block_sum64(ws, red);
+    ftok = block_sum64(ftok, red);
+    int32_t split_s = A.split_opt;
+    if (split_s <= 0) {
+        const int64_t t = ws * A.Hkv / (int64_t)(32 * max(1, A.num_sms));
+        split_s = (int32_t)min((int64_t)8192, max((int64_t)kMinOwnChunk, (t + 63) / 64 * 64));
+    }
+    for (int32_t b = threadIdx.x; b < kBins; b += blockDim.x) bins[b] = 0;
+    __syncthreads();
+    for (int32_t r = threadIdx.x; r < R; r += blockDim.x) {
+        const int32_t tok = A.seq_lens[r] - A.suffix_start[r] * kBlockSize;
+        const int32_t nch = (tok + split_s - 1) / split_s;
+        const int32_t chunk = nch ? ((tok + nch - 1) / nch + kBlockSize - 1) / kBlockSize * kBlockSize : 0;
+        A.nch[r] = nch;
+        A.chunk[r] = chunk;
+        if (nch) {
+            const int32_t last = tok - (nch - 1) * chunk;
+            atomicAdd(&bins[length_bin(chunk)], A.Hkv * (nch - 1));
+            atomicAdd(&bins[length_bin(last)], A.Hkv);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int32_t acc = 0;
+        for (int32_t b = kBins - 1; b >= 0; --b) {
+            A.bin_cursor[b] = acc;
+            acc += bins[b];
+        }
+    }
+    __syncthreads();
+    const int64_t n_sitems = block_exclusive_scan(R, [&](int32_t r) { return (int64_t)A.Hkv * A.nch[r]; },
+                                                  A.s_item_off, red);
+    const int64_t n_spart = block_exclusive_scan(
+        R, [&](int32_t r) { return (int64_t)A.Hkv * A.nch[r] * G; }, A.part, red);
+    for (int32_t r = threadIdx.x; r < R; r += blockDim.x) A.part[r] += (int32_t)A.n_ppart;
+    if (threadIdx.x == 0) {
+        hdr->split_tokens = split_s;
+        hdr->n_suffix_items = (int32_t)n_sitems;
+        hdr->n_suffix_partials = (int32_t)n_spart;
+        hdr->suffix_tok_sum = ws;
+        hdr->flat_kv_tokens = ftok;
+    }
+}
+
 // ------------------------------------------------------------ host helpers
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -1048,6 +1139,8 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
         }
         P->dev_allocs.push_back(base);
         P->workspace_bytes += wa.bytes;
+        P->cap_suffix_items = H.n_suffix_items;
+        P->cap_partials = n_part;
     }
 
     if (!flat && H.n_groups > 0) {
@@ -1073,6 +1166,128 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
             R, P->seq_lens, P->suffix_start, P->s_nch, P->s_chunk, P->s_part, bin_cursor, G, Hkv, P->suffix_items);
         FCA_CK(cudaGetLastError());
     }
+    return FCA_OK;   // temporaries go back to the pool in stream order
+}
+
+// Next decode step of the same batch: new lengths (and tables grown past the
+// blocks the plan's groups read) over the plan's forest.  Everything is
+// checked before the plan changes; on an error return it is as it was.
+fca_status plan_update(const int32_t* block_tables, const int32_t* seq_lens, cudaStream_t stream,
+                       fca_plan_s* P) {
+    const int32_t R = P->R, max_blocks = P->max_blocks, num_blocks = P->num_blocks;
+    const int32_t Hkv = P->Hkv, D = P->D, G = P->G;
+
+    int32_t* valid = nullptr;
+    int32_t* nfull = nullptr;
+    PlanHeader* hdr = nullptr;
+    int32_t* t_nch = nullptr;
+    int32_t* t_chunk = nullptr;
+    int32_t* t_part = nullptr;
+    int32_t* t_item_off = nullptr;
+    int32_t* bin_cursor = nullptr;
+    Arena ta;
+    ta.add(&valid, num_blocks);
+    ta.add(&hdr, 1);
+    const size_t zero1 = ta.bytes;
+    ta.add(&nfull, R);
+    ta.add(&t_nch, R);
+    ta.add(&t_chunk, R);
+    ta.add(&t_part, R + 1);
+    ta.add(&t_item_off, R + 1);
+    ta.add(&bin_cursor, kBins);
+    TempArena tmp(stream);
+    if (ta.commit(stream, &tmp.base) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return FCA_ERR_OOM;
+    }
+    FCA_CK(cudaMemsetAsync(tmp.base, 0, zero1, stream));
+    const int64_t cells = (int64_t)R * max_blocks;
+    k_validate<<<grid_for(cells, 256), 256, 0, stream>>>(block_tables, max_blocks, seq_lens, R, num_blocks, nfull,
+                                                          valid, hdr);
+    k_check_shared<<<grid_for(cells, 256), 256, 0, stream>>>(block_tables, seq_lens, P->bt, P->suffix_start, R,
+                                                             max_blocks, hdr);
+    k_unique_tokens<<<grid_for(num_blocks, 256), 256, 0, stream>>>(valid, num_blocks, hdr);
+    FCA_CK(cudaGetLastError());
+    UpdateOwnArgs ua{};
+    ua.R = R;
+    ua.Hkv = Hkv;
+    ua.G = G;
+    ua.split_opt = P->opts.split_tokens;
+    {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        ua.num_sms = 148;
+        cudaDeviceGetAttribute(&ua.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    ua.n_ppart = P->hdr.n_prefix_partials;
+    ua.seq_lens = seq_lens;
+    ua.suffix_start = P->suffix_start;
+    ua.nch = t_nch;
+    ua.chunk = t_chunk;
+    ua.part = t_part;
+    ua.s_item_off = t_item_off;
+    ua.bin_cursor = bin_cursor;
+    ua.hdr = hdr;
+    const size_t upd_smem = (64 + 1024) * 8 + kBins * 4;
+    k_update_own<<<1, 1024, upd_smem, stream>>>(ua);
+    FCA_CK(cudaGetLastError());
+
+    PlanHeader H{};
+    FCA_CK(cudaMemcpyAsync(&H, hdr, sizeof(PlanHeader), cudaMemcpyDeviceToHost, stream));
+    FCA_CK(cudaStreamSynchronize(stream));
+    if (H.status & kPlanBadSeqLen) return FCA_ERR_INVALID_ARG;
+    if (H.status & kPlanBadBlockId) return FCA_ERR_BAD_BLOCK_ID;
+    if (H.status & kPlanUpdateMismatch) return FCA_ERR_INVALID_ARG;
+    const int64_t n_part = (int64_t)P->hdr.n_prefix_partials + H.n_suffix_partials;
+    if (n_part >= (int64_t)INT32_MAX / 2) return FCA_ERR_UNSUPPORTED;
+
+    // more own work than the plan has room for: a new block for the own-pass
+    // items and every partial row (the grouped pass's rows are rewritten by
+    // each decode, so nothing needs copying)
+    if (H.n_suffix_items > P->cap_suffix_items || n_part > P->cap_partials) {
+        const int64_t items = std::max<int64_t>(H.n_suffix_items, P->cap_suffix_items) * 5 / 4 + 64;
+        const int64_t rows = std::max<int64_t>(n_part, P->cap_partials) * 5 / 4 + 64;
+        SuffixItem* n_items = nullptr;
+        float* n_lse = nullptr;
+        float* n_o = nullptr;
+        Arena na;
+        na.add(&n_items, (size_t)items);
+        na.add(&n_lse, (size_t)rows);
+        na.add(&n_o, (size_t)rows * D);
+        void* base = nullptr;
+        if (na.commit(stream, &base) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return FCA_ERR_OOM;
+        }
+        P->dev_allocs.push_back(base);
+        P->workspace_bytes += na.bytes;
+        P->suffix_items = n_items;
+        P->part_lse = n_lse;
+        P->part_o = n_o;
+        P->cap_suffix_items = items;
+        P->cap_partials = rows;
+    }
+
+    // apply: the new tables and lengths, the own-pass arrays, the item list
+    FCA_CK(cudaMemcpyAsync(P->bt, block_tables, (size_t)cells * sizeof(int32_t), cudaMemcpyDeviceToDevice, stream));
+    FCA_CK(cudaMemcpyAsync(P->seq_lens, seq_lens, (size_t)R * sizeof(int32_t), cudaMemcpyDeviceToDevice, stream));
+    FCA_CK(cudaMemcpyAsync(P->s_nch, t_nch, (size_t)R * sizeof(int32_t), cudaMemcpyDeviceToDevice, stream));
+    FCA_CK(cudaMemcpyAsync(P->s_chunk, t_chunk, (size_t)R * sizeof(int32_t), cudaMemcpyDeviceToDevice, stream));
+    FCA_CK(cudaMemcpyAsync(P->s_part, t_part, (size_t)(R + 1) * sizeof(int32_t), cudaMemcpyDeviceToDevice, stream));
+    if (H.n_suffix_items > 0) {
+        k_fill_suffix_items<<<grid_for(R, 128), 128, 0, stream>>>(R, P->seq_lens, P->suffix_start, P->s_nch,
+                                                                  P->s_chunk, P->s_part, bin_cursor, G, Hkv,
+                                                                  P->suffix_items);
+        FCA_CK(cudaGetLastError());
+    }
+    PlanHeader& PH = P->hdr;
+    PH.split_tokens = H.split_tokens;
+    PH.n_suffix_items = H.n_suffix_items;
+    PH.n_suffix_partials = H.n_suffix_partials;
+    PH.suffix_tok_sum = H.suffix_tok_sum;
+    PH.flat_kv_tokens = H.flat_kv_tokens;
+    PH.unique_kv_tokens = H.unique_kv_tokens;
+    PH.fca_kv_tokens = PH.prefix_tok_sum + H.suffix_tok_sum;
     return FCA_OK;   // temporaries go back to the pool in stream order
 }
 

@@ -491,3 +491,196 @@ def test_parent_folded_into_child_items(cover):
         assert st["prefix_items"] >= 5
     o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
     assert_close(o, l, o_ref, l_ref, f"fold-in cover={cover}")
+
+
+# --------------------------------------------------------------- plan update
+
+def pooled(w, extra_blocks, max_blocks, seed):
+    """w with its K/V cache inside a pool of extra_blocks more blocks (their
+    K/V drawn fresh, free for later tokens) and its tables widened to
+    max_blocks columns, as an engine with a block pool keeps a batch."""
+    shape = (extra_blocks, w.block_size, w.Hkv, w.D)
+    kc = np.concatenate([w.k_cache, fca_workloads.normal_bf16(shape, seed, 11)])
+    vc = np.concatenate([w.v_cache, fca_workloads.normal_bf16(shape, seed, 12)])
+    bt = np.zeros((w.R, max_blocks), np.int32)
+    bt[:, :w.max_blocks] = w.block_tables
+    return fca_workloads.Workload(w.name, w.q, kc, vc, bt, w.seq_lens.copy(), w.Hq, w.Hkv, w.D,
+                                  w.block_size, w.seed)
+
+
+def grown(w, extra, first_free, seed):
+    """The batch w after request r has extra[r] more tokens: they go first into
+    r's last block (always private: a shared prompt's partial tail is a private
+    copy) and then into new blocks taken in turn from first_free on.  Same pool,
+    same table width, new queries."""
+    B = w.block_size
+    sl = (w.seq_lens.astype(np.int64) + np.asarray(extra, np.int64)).astype(np.int32)
+    bt = w.block_tables.copy()
+    nxt = first_free
+    for r in range(w.R):
+        for j in range((int(w.seq_lens[r]) + B - 1) // B, (int(sl[r]) + B - 1) // B):
+            bt[r, j] = nxt
+            nxt += 1
+    assert nxt <= w.num_blocks and bt.shape[1] * B >= sl.max()
+    q = fca_workloads.normal_bf16(w.q.shape, seed, 13)
+    return fca_workloads.Workload(w.name + "+", q, w.k_cache, w.v_cache, bt, sl, w.Hq, w.Hkv, w.D, B, w.seed)
+
+
+def decode_with(plan, w, flat=False):
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    q, k, v, _, _ = w.torch_inputs("cuda")
+    out = torch.empty_like(q)
+    lse = torch.empty(w.R, w.Hq, dtype=torch.float32, device="cuda")
+    (fca.fca_flat_decode if flat else fca.fca_decode)(q, k, v, plan, out, lse, w.scale)
+    assert fca.fca_check_device_status(plan) == 0
+    return out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def check_all(plan, w, what, flat=False):
+    o, l = decode_with(plan, w, flat)
+    o_ref, l_ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    assert_close(o, l, o_ref, l_ref, what)
+
+
+def growth_steps(w0, seed, n_steps=4, most=80):
+    """w0 in a pool with room for n_steps steps of 1..most tokens a request,
+    and the batch after each step."""
+    rng = np.random.default_rng(500 + seed)
+    steps = [rng.integers(1, most + 1, size=w0.R) for _ in range(n_steps)]
+    B = w0.block_size
+    final = w0.seq_lens.astype(np.int64) + np.sum(steps, axis=0)
+    need = int(((final + B - 1) // B - (w0.seq_lens.astype(np.int64) + B - 1) // B).sum())
+    base = pooled(w0, need, int(((final + B - 1) // B).max()), seed)
+    out, cur = [], base
+    for ex in steps:
+        # each step's new blocks follow the ones taken before
+        used = int(((cur.seq_lens.astype(np.int64) + B - 1) // B).sum()
+                   - ((w0.seq_lens.astype(np.int64) + B - 1) // B).sum())
+        cur = grown(cur, ex, w0.num_blocks + used, seed + len(out))
+        out.append(cur)
+    return base, out
+
+
+@pytest.mark.parametrize("seed", range(10))
+@pytest.mark.parametrize("split", [0, 64])
+def test_plan_update_follows_growing_requests(seed, split):
+    # one plan kept over four decode steps: after each step every request has
+    # grown by 1-80 tokens (some into new blocks); the updated plan decodes like
+    # attention over the new tables and holds the forest the oracle finds in
+    # them.  A split of 64 tokens makes the own-pass work outgrow the plan's
+    # first allocation.
+    import shared_prefix_kv_fca_b200 as fca
+    w0 = fca_workloads.random_small(seed, max_requests=24)
+    base, steps = growth_steps(w0, seed)
+    bt, sl = base.torch_inputs("cuda")[3:]
+    ref = oracle.plan(base.block_tables, base.seq_lens, 16)
+    with fca.fca_plan(bt, sl, base.num_blocks, w0.Hq, w0.Hkv, w0.D, min_saved_blocks=0,
+                      split_tokens=split) as plan:
+        assert_plan_equal(plan.export(), ref)
+        check_all(plan, base, f"seed {seed} step 0")
+        for s, cur in enumerate(steps):
+            bt2, sl2 = cur.torch_inputs("cuda")[3:]
+            plan.update(bt2, sl2)
+            exp = plan.export()
+            assert_plan_equal(exp, oracle.plan(cur.block_tables, cur.seq_lens, 16))
+            assert_plan_equal(exp, ref)
+            st = plan.stats()
+            assert st["unique_kv_tokens"] == oracle.unique_kv_tokens(cur.block_tables, cur.seq_lens, 16,
+                                                                       cur.num_blocks)
+            check_all(plan, cur, f"seed {seed} step {s + 1}")
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_plan_update_flat(seed):
+    import shared_prefix_kv_fca_b200 as fca
+    w0 = fca_workloads.random_small(seed, max_requests=24)
+    base, steps = growth_steps(w0, seed, n_steps=2)
+    bt, sl = base.torch_inputs("cuda")[3:]
+    with fca.fca_plan(bt, sl, base.num_blocks, w0.Hq, w0.Hkv, w0.D, flat=True) as plan:
+        check_all(plan, base, f"flat seed {seed} step 0", flat=True)
+        for s, cur in enumerate(steps):
+            bt2, sl2 = cur.torch_inputs("cuda")[3:]
+            plan.update(bt2, sl2)
+            assert plan.stats()["num_groups"] == 0
+            check_all(plan, cur, f"flat seed {seed} step {s + 1}", flat=True)
+
+
+def test_plan_update_refusals_leave_the_plan_usable():
+    # tables that no longer fit the plan's forest are refused with a status,
+    # and the plan still decodes the batch it was built or last updated for
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    for seed in range(40):
+        w0 = fca_workloads.random_small(seed, max_requests=24)
+        ref = oracle.plan(w0.block_tables, w0.seq_lens, 16)
+        if w0.R >= 2 and ref["suffix_start"].max() > 1:
+            break
+    base, (nxt,) = growth_steps(w0, seed, n_steps=1)
+    r = int(np.argmax(ref["suffix_start"]))
+    ss = int(ref["suffix_start"][r])
+    B = 16
+
+    def attempt(bt_np, sl_np):
+        bt_t = torch.from_numpy(np.ascontiguousarray(bt_np, np.int32)).cuda()
+        sl_t = torch.from_numpy(np.ascontiguousarray(sl_np, np.int32)).cuda()
+        with pytest.raises(fca.FcaError) as ei:
+            plan.update(bt_t, sl_t)
+        return ei.value.status
+
+    bt, sl = base.torch_inputs("cuda")[3:]
+    with fca.fca_plan(bt, sl, base.num_blocks, w0.Hq, w0.Hkv, w0.D, min_saved_blocks=0) as plan:
+        bad = nxt.block_tables.copy()
+        bad[r, ss - 1] = base.num_blocks - 1          # a shared entry replaced
+        assert attempt(bad, nxt.seq_lens) == 1
+        short = nxt.seq_lens.copy()
+        short[r] = ss * B - 1                        # the request no longer covers its groups
+        assert attempt(nxt.block_tables, short) == 1
+        assert attempt(nxt.block_tables[:-1], nxt.seq_lens[:-1]) == 1    # a request fewer
+        wide = np.zeros((nxt.R, nxt.max_blocks + 1), np.int32)
+        wide[:, :-1] = nxt.block_tables
+        assert attempt(wide, nxt.seq_lens) == 1                          # another table width
+        oob = nxt.block_tables.copy()
+        last = (int(nxt.seq_lens[r]) + B - 1) // B - 1
+        oob[r, last] = base.num_blocks                # a used entry outside the pool
+        assert attempt(oob, nxt.seq_lens) == 2
+        too_long = nxt.seq_lens.copy()
+        too_long[r] = nxt.max_blocks * B + 1
+        assert attempt(nxt.block_tables, too_long) == 1
+        assert_plan_equal(plan.export(), ref)
+        check_all(plan, base, "after refused updates")
+        bt2, sl2 = nxt.torch_inputs("cuda")[3:]
+        plan.update(bt2, sl2)
+        check_all(plan, nxt, "after the good update")
+
+
+def test_plan_update_full_size_one_token_steps():
+    # the decode loop on the llama8b workload: every request gains one token a
+    # step for 20 steps (some cross into new blocks); one plan, updated each step
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    w0 = fca_workloads.make("llama8b")
+    B = 16
+    n_steps = 20
+    final = w0.seq_lens.astype(np.int64) + n_steps
+    need = int(((final + B - 1) // B - (w0.seq_lens.astype(np.int64) + B - 1) // B).sum())
+    base = pooled(w0, need, int(((final + B - 1) // B).max()), 0)
+    q, k, v, bt, sl = base.torch_inputs("cuda")
+    cur = base
+    with fca.fca_plan(bt, sl, base.num_blocks, w0.Hq, w0.Hkv, w0.D) as plan:
+        ref = plan.export()
+        taken = 0
+        for s in range(n_steps):
+            nb_before = (cur.seq_lens.astype(np.int64) + B - 1) // B
+            cur = grown(cur, np.ones(w0.R, np.int64), w0.num_blocks + taken, s)
+            taken += int(((cur.seq_lens.astype(np.int64) + B - 1) // B - nb_before).sum())
+            bt2, sl2 = cur.torch_inputs("cuda")[3:]
+            plan.update(bt2, sl2)
+        assert_plan_equal(plan.export(), ref)
+        assert_plan_equal(ref, oracle.plan(cur.block_tables, cur.seq_lens, 16, min_saved_blocks=32))
+        o, l = decode_with(plan, cur)
+    pairs = sampled_pairs(cur, 48)
+    o_ref, l_ref = oracle.paged_attention(cur.q, cur.k_cache, cur.v_cache, cur.block_tables, cur.seq_lens,
+                                          cur.scale, pairs=pairs)
+    sel = (pairs[:, 0], pairs[:, 1])
+    assert_close(o[sel], l[sel], o_ref, l_ref, "llama8b after 20 updates")
