@@ -135,6 +135,10 @@ fca_status fca_plan(const int32_t *block_tables, int32_t max_blocks, const int32
  *                 blocks (the ones its groups read) must be unchanged and its
  *                 seq_len must still cover them.
  *
+ * The plan's tables, lengths and own-pass work lists are rewritten on
+ * `stream`: call it on the stream the plan's decodes use, after the decode
+ * of the previous step has been queued there.
+ *
  * Synchronises `stream` once (the new sizes), like fca_plan; may take more
  * memory from the plan pool if the own work outgrew the plan.  Errors:
  * FCA_ERR_INVALID_ARG (a shared entry changed, a length no longer covers the
