@@ -225,6 +225,17 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def unique_bytes(w) -> int:
     import oracle
     return oracle.unique_kv_tokens(w.block_tables, w.seq_lens, w.block_size, w.num_blocks) * w.Hkv * w.D * 4
@@ -251,6 +262,7 @@ def reference_arm(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload_desc(w)}, "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+                             "cpu_model": cpu_model(),
                              "sample": f"whole requests (all {w.Hq} heads) totalling about "
                                        f"{per_step_budget:.1f} s of CPU work per step, time scaled "
                                        f"to the full batch of {total_tok} tokens"},
@@ -318,12 +330,13 @@ def fca_arm(args):
     flat_plan = None if args.no_flat else fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, flat=True,
                                                        split_tokens=args.split)
 
-    def run_steps(p, n, timed):
+    def run_steps(p, n, timed, flush_l2=True):
         """n whole decode steps (fca_decode: both passes side by side, then the
         merge), each bracketed by events on the launching stream."""
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         for i in range(n):
-            flush.zero_()
+            if flush_l2:
+                flush.zero_()
             ev[i][0].record(stream)
             fca.fca_decode(q, k, v, p, out, lse, w.scale, stream)
             ev[i][1].record(stream)
@@ -386,6 +399,12 @@ def fca_arm(args):
     assert fca.fca_check_device_status(plan, stream) == 0
     step_ms, total_unique, value = aggregate_step(step_ms_rank, st["unique_kv_bytes"], red)
     n_launch = (1 if (st["prefix_items"] > 0) else 0) + (1 if st["suffix_items"] > 0 else 0) + 1
+
+    # ---- the same steps back to back without the L2 flush (warm L2)
+    run_steps(plan, args.warmup, False, flush_l2=False)
+    barrier()
+    warm_ms = max_over_ranks(run_steps(plan, args.steps, True, flush_l2=False))
+    barrier()
 
     # ---- the passes one at a time (per-kernel roofline)
     run_passes(plan, args.warmup, False)
@@ -547,9 +566,21 @@ def fca_arm(args):
             sec, tok, nreq = oracle_sample(w, args.cpu_budget_s)
             full_s = sec * float(w.seq_lens.sum()) / tok
             cpu = {"value": st["unique_kv_bytes"] / full_s / 1e9, "unit": "GB/s", "cores": cpu_cores(),
-                   "kind": "oracle", "ms_per_step": full_s * 1e3,
+                   "kind": "oracle", "ms_per_step": full_s * 1e3, "cpu_model": cpu_model(),
                    "sample": f"{nreq} whole requests x {w.Hq} heads ({tok} tokens of "
                              f"{int(w.seq_lens.sum())}) in {sec:.1f} s, scaled to the full batch"}
+            # the same oracle on one core, a smaller sample
+            import oracle
+            before = oracle.set_threads(1)
+            try:
+                sec1, tok1, nreq1 = oracle_sample(w, args.cpu_budget_s / 4, seed=1)
+            finally:
+                oracle.set_threads(before)
+            full1 = sec1 * float(w.seq_lens.sum()) / tok1
+            cpu["one_core"] = {"value": st["unique_kv_bytes"] / full1 / 1e9, "unit": "GB/s", "cores": 1,
+                               "ms_per_step": full1 * 1e3,
+                               "sample": f"{nreq1} whole requests x {w.Hq} heads ({tok1} tokens) in "
+                                         f"{sec1:.1f} s, scaled to the full batch"}
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "us_per_step": step_ms * 1e3,
@@ -561,6 +592,7 @@ def fca_arm(args):
                        "flat_kv_bytes_per_rank": st["flat_kv_bytes"], "replicas": world},
             "pct_of_peak": 100.0 * value / (peak * world), "peak_gbs": peak, "peak_kind": peak_kind,
             "plan_ms": plan_ms,
+            "warm_l2_us_per_step": warm_ms * 1e3,
             "passes_us": {key: val * 1e3 for key, val in pass_ms.items()},
             "serial_passes_us_per_step": serial_ms * 1e3,
             "flat_us_per_step": flat_ms * 1e3 if flat_ms else None,

@@ -69,8 +69,16 @@ def _load():
         lib.oracle_unique_kv_tokens.argtypes = [i32p, ctypes.c_int32, ctypes.c_int32, i32p,
                                                 ctypes.c_int32, ctypes.c_int64]
         lib.oracle_unique_kv_tokens.restype = ctypes.c_int64
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
+
+
+def set_threads(n: int) -> int:
+    """Threads of paged_attention's parallel loop (for timing; the result does
+    not depend on it); n <= 0 leaves it.  Returns the count in force before."""
+    return int(_load().oracle_set_threads(int(n)))
 
 
 def _bits(a) -> np.ndarray:

@@ -48,6 +48,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORACLE_OK 0
 #define ORACLE_ERR_ARG -1
@@ -455,4 +458,19 @@ int64_t oracle_unique_kv_tokens(const int32_t *block_tables, int32_t R, int32_t 
     for (int64_t b = 0; b < num_blocks; ++b) total += valid[b];
     free(valid);
     return total;
+}
+
+/* Threads of the OpenMP loop in oracle_paged_attention (timing only; the
+ * result does not depend on it).  Returns the count in force before. */
+int oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    int before = omp_get_max_threads();
+    if (n > 0)
+        omp_set_num_threads(n);
+    return before;
+#else
+    (void)n;
+    return 1;
+#endif
 }

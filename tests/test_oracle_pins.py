@@ -428,3 +428,17 @@ def test_kv_bytes_per_token_worked_example():
     assert per_token_layer * g["layers"] == g["page_bytes_per_token_kib"] * 1024
     total_kib = g["page_context_tokens"] * per_token_layer * g["layers"] / 1024
     assert total_kib == 12.8e6
+
+
+def test_oracle_attention_independent_of_thread_count():
+    # the CPU baseline times the oracle on all cores and on one; each
+    # (request, head) is computed alone, so the results are bit-identical
+    w = fca_workloads.random_small(3, max_requests=12)
+    before = oracle.set_threads(1)
+    try:
+        o1, l1 = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    finally:
+        oracle.set_threads(before)
+    on, ln = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    np.testing.assert_array_equal(o1, on)
+    np.testing.assert_array_equal(l1, ln)
