@@ -33,7 +33,7 @@ def test_header_declares_the_expected_entry_points():
     names = declared_functions()
     for n in ["fca_plan", "fca_decode", "fca_flat_decode", "fca_plan_get_stats", "fca_plan_export",
               "fca_plan_member_count", "fca_plan_destroy", "fca_check_device_status",
-              "fca_status_string", "fca_version", "fca_plan_opts_default"]:
+              "fca_status_string", "fca_version", "fca_plan_opts_default", "fca_plan_update"]:
         assert n in names
 
 
@@ -82,3 +82,7 @@ def test_argument_checks_return_status_without_a_device(lib):
     assert lib.fca_decode(fake, fake, fake, None, fake, None, 0.1, None) == 1
     assert lib.fca_flat_decode(fake, fake, fake, None, fake, None, 0.1, None) == 1
     assert lib.fca_plan_destroy(None) == 0
+    # update without a plan, or without tables
+    assert lib.fca_plan_update(None, fake, 4, fake, 2, None) == 1
+    assert lib.fca_plan_update(fake, None, 4, fake, 2, None) == 1
+    assert lib.fca_plan_update(fake, fake, 4, None, 2, None) == 1
