@@ -250,6 +250,21 @@ fca_status fca_plan_destroy(fca_plan_t plan);
 fca_status fca_check_device_status(fca_plan_t plan, void *stream, int32_t *code);
 
 /*
+ * fca_selftest_wait_timeout -- check that a wait which runs out ends in a
+ * status, not a hang.  Every spin-wait of this library's kernels is bounded
+ * by 1 s of wall-clock time; when the bound is reached the kernel records
+ * bit 1 in a device error word and returns.  This call runs one
+ * single-thread kernel whose wait, through the same bounded wait, is for a
+ * barrier phase that nothing completes, and copies the error word it
+ * recorded into *out_word (HOST): bit 1 set means the wait gave up as
+ * designed.  Takes about 1 s; synchronises `stream`; uses the current
+ * device.  Returns FCA_OK when the kernel ran, FCA_ERR_INVALID_ARG for a
+ * NULL out_word, FCA_ERR_OOM / FCA_ERR_CUDA when a CUDA call failed.  Not a
+ * step of the method: a diagnostic of its failure detection.
+ */
+fca_status fca_selftest_wait_timeout(void *stream, int32_t *out_word);
+
+/*
  * fca_paged_decode_static -- the flat paged decode of fca_flat_decode
  * (standard split-KV attention of every request over its whole block table,
  * then the log-sum-exp merge) in one call that allocates nothing.  This entry

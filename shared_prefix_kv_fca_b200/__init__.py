@@ -105,6 +105,8 @@ def load_library():
     lib.fca_plan_member_count.argtypes = [vp, ctypes.POINTER(ctypes.c_int64)]
     lib.fca_plan_member_count.restype = ctypes.c_int
     lib.fca_plan_update.argtypes = [vp, vp, i32, vp, i32, vp]
+    lib.fca_selftest_wait_timeout.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.fca_selftest_wait_timeout.restype = ctypes.c_int
     lib.fca_plan_update.restype = ctypes.c_int
     lib.fca_plan_destroy.argtypes = [vp]
     lib.fca_plan_destroy.restype = ctypes.c_int
@@ -302,6 +304,15 @@ def fca_check_device_status(plan: "Plan", stream=None) -> int:
     if rc == 6:
         raise FcaError(rc, f"fca_check_device_status (word {code.value:#x})")
     return int(code.value)
+
+
+def fca_selftest_wait_timeout(stream=None) -> int:
+    """Run the kernel whose bounded wait is made to run out; return the device
+    error word it recorded (bit 1: the wait gave up after its 1 s bound)."""
+    word = ctypes.c_int32()
+    _check(load_library().fca_selftest_wait_timeout(_stream_handle(stream), ctypes.byref(word)),
+           "fca_selftest_wait_timeout")
+    return int(word.value)
 
 
 def fca_plan_destroy(plan: "Plan") -> None:

@@ -17,7 +17,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libfca_b200.so")
-SOURCES = ["fca_api.cu", "fca_plan.cu", "fca_suffix.cu", "fca_prefix.cu", "fca_merge.cu", "fca_static.cu"]
+SOURCES = ["fca_api.cu", "fca_plan.cu", "fca_suffix.cu", "fca_prefix.cu", "fca_merge.cu", "fca_static.cu",
+           "fca_selftest.cu"]
 HEADERS = ["fca_internal.h", "fca_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -82,7 +82,20 @@ def test_argument_checks_return_status_without_a_device(lib):
     assert lib.fca_decode(fake, fake, fake, None, fake, None, 0.1, None) == 1
     assert lib.fca_flat_decode(fake, fake, fake, None, fake, None, 0.1, None) == 1
     assert lib.fca_plan_destroy(None) == 0
+    # the wait self-test without somewhere to put the word
+    assert lib.fca_selftest_wait_timeout(None, None) == 1
     # update without a plan, or without tables
     assert lib.fca_plan_update(None, fake, 4, fake, 2, None) == 1
     assert lib.fca_plan_update(fake, None, 4, fake, 2, None) == 1
     assert lib.fca_plan_update(fake, fake, 4, None, 2, None) == 1
+
+
+def test_selftest_binding_without_a_device(lib):
+    # the binding's whole path up to the first CUDA call, which fails here
+    # (no device); on a GPU machine the gpu-marked test runs the kernel itself
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present: tests/test_gpu_failure_detection.py covers the call")
+    with pytest.raises(fca.FcaError) as ei:
+        fca.fca_selftest_wait_timeout(stream=0)
+    assert ei.value.status == 4
