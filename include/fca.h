@@ -142,8 +142,10 @@ fca_status fca_plan(const int32_t *block_tables, int32_t max_blocks, const int32
  * Synchronises `stream` once (the new sizes), like fca_plan; may take more
  * memory from the plan pool if the own work outgrew the plan.  Errors:
  * FCA_ERR_INVALID_ARG (a shared entry changed, a length no longer covers the
- * shared blocks or is out of range), FCA_ERR_BAD_BLOCK_ID, FCA_ERR_CUDA,
- * FCA_ERR_OOM; on an error the plan is left as it was.  Not part of the
+ * shared blocks or is out of range, another table shape), FCA_ERR_BAD_BLOCK_ID,
+ * FCA_ERR_UNSUPPORTED (more partial rows than the planner indexes),
+ * FCA_ERR_OOM, FCA_ERR_CUDA.  After any of them but FCA_ERR_CUDA the plan is
+ * left as it was; after FCA_ERR_CUDA destroy it.  Not part of the
  * method's steps: it is "Core Mechanism" step 1 carried over from one decode
  * step to the next.
  */
