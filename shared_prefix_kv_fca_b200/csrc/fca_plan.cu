@@ -1197,6 +1197,7 @@ fca_status plan_update(const int32_t* block_tables, const int32_t* seq_lens, cud
     ta.add(&bin_cursor, kBins);
     TempArena tmp(stream);
     if (ta.commit(stream, &tmp.base) != cudaSuccess) {
+        tmp.base = nullptr;
         (void)cudaGetLastError();
         return FCA_ERR_OOM;
     }
