@@ -390,8 +390,10 @@ def fca_arm(args):
     keep_busy(0.6)   # every rank, so that the ranks' timed regions run at the same time
     barrier()
     torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_push("fca_decode: timed steps")
     step_ms_rank = run_steps(plan, args.steps, True)
     torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_pop()
     barrier()
     keep_busy(0.6)
     clocks = sampler.stop() if sampler else None
@@ -409,7 +411,9 @@ def fca_arm(args):
     # ---- the passes one at a time (per-kernel roofline)
     run_passes(plan, args.warmup, False)
     barrier()
+    torch.cuda.nvtx.range_push("passes one at a time: timed steps")
     fca_t = run_passes(plan, args.steps, True)
+    torch.cuda.nvtx.range_pop()
     barrier()
     assert fca.fca_check_device_status(plan, stream) == 0
 
@@ -418,7 +422,10 @@ def fca_arm(args):
     if flat_plan is not None:
         run_steps(flat_plan, args.warmup, False)
         barrier()
-        flat_ms = max_over_ranks(run_steps(flat_plan, args.steps, True))
+        torch.cuda.nvtx.range_push("flat decode: timed steps")
+        flat_ms_rank = run_steps(flat_plan, args.steps, True)
+        torch.cuda.nvtx.range_pop()
+        flat_ms = max_over_ranks(flat_ms_rank)
         barrier()
         assert fca.fca_check_device_status(flat_plan, stream) == 0
 
