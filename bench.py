@@ -114,30 +114,53 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.out.close()
-        rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+            lines = f.readlines()
         os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = set()
-        for r in rows:
-            for name, val in zip(names, r[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        busy = [s for s, p in zip(sm, pw) if p >= 200.0]
-        loaded = busy or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(busy),
-                "power_w_max": max(pw) if pw else None}
+        return summarize_clock_samples(lines)
+
+
+def _num(text: str):
+    try:
+        return float(text)
+    except ValueError:
+        return None
+
+
+def summarize_clock_samples(lines, busy_watts: float = 200.0):
+    """Summary of nvidia-smi rows in ClockSampler.FIELDS order (csv, no header,
+    no units): the median SM clock over the samples drawn under load (power at
+    least busy_watts; all samples if none was), the highest max clock, the
+    throttle reasons seen active in any sample, and the sample counts.  Fields
+    that are not numbers ("[N/A]") leave their sample out of that statistic."""
+    rows = []
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) >= 9:
+            rows.append(parts)
+    if not rows:
+        return None
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = set()
+    sm, mx, pw, busy = [], [], [], []
+    for r in rows:
+        s_mhz, m_mhz, watts = _num(r[1]), _num(r[2]), _num(r[3])
+        if s_mhz is not None:
+            sm.append(s_mhz)
+            if watts is not None and watts >= busy_watts:
+                busy.append(s_mhz)
+        if m_mhz is not None:
+            mx.append(m_mhz)
+        if watts is not None:
+            pw.append(watts)
+        for name, val in zip(names, r[5:9]):
+            if val.lower() == "active":
+                reasons.add(name)
+    loaded = busy or sm
+    return {"sm_mhz": statistics.median(loaded) if loaded else None,
+            "sm_max_mhz": max(mx) if mx else None,
+            "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(busy),
+            "power_w_max": max(pw) if pw else None}
 
 
 def gpu_id_for(local_rank: int) -> str:
