@@ -138,6 +138,38 @@ def _stream_handle(stream) -> Optional[int]:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _check_tables(block_tables, seq_lens) -> None:
+    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens")):
+        if not t.is_cuda or str(t.dtype) != "torch.int32" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    if block_tables.dim() != 2 or tuple(seq_lens.shape) != (block_tables.shape[0],):
+        raise ValueError("block_tables must be [R, max_blocks] and seq_lens [R]")
+
+
+def _check_bf16(t, name: str, shape=None) -> None:
+    if not t.is_cuda or str(t.dtype) != "torch.bfloat16" or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+
+
+def _check_caches(k_cache, v_cache, num_blocks: int, Hkv: int, D: int) -> None:
+    """The kernels read num_blocks x 16 x Hkv x D elements of each cache."""
+    for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check_bf16(t, name)
+        if t.dim() != 4 or tuple(t.shape[1:]) != (16, Hkv, D) or t.shape[0] < num_blocks:
+            raise ValueError(f"{name} must be [>= {num_blocks}, 16, {Hkv}, {D}], not {tuple(t.shape)}")
+
+
+def _check_lse(lse, R: int, Hq: int) -> None:
+    if lse is None:
+        return
+    if not lse.is_cuda or str(lse.dtype) != "torch.float32" or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 CUDA tensor")
+    if tuple(lse.shape) != (R, Hq):
+        raise ValueError(f"lse must have shape {(R, Hq)}, not {tuple(lse.shape)}")
+
+
 def _check(rc: int, where: str) -> None:
     if rc != 0:
         raise FcaError(rc, where)
@@ -170,9 +202,7 @@ def fca_plan(block_tables, seq_lens, num_blocks: int, num_q_heads: int, num_kv_h
     sharing saves fewer block reads ((members - 1) x length in blocks) are
     folded (0 keeps every shared prefix)."""
     lib = load_library()
-    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens")):
-        if not t.is_cuda or str(t.dtype) != "torch.int32" or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    _check_tables(block_tables, seq_lens)
     R, mb = block_tables.shape
     o = fca_plan_opts(min_group_size, min_shared_blocks, split_tokens, FCA_PLAN_FLAT if flat else 0,
                       min_saved_blocks)
@@ -181,18 +211,18 @@ def fca_plan(block_tables, seq_lens, num_blocks: int, num_q_heads: int, num_kv_h
                       num_kv_heads, head_dim, ctypes.byref(o), ctypes.byref(handle),
                       _stream_handle(stream))
     _check(rc, "fca_plan")
-    return Plan(handle, R, num_q_heads, num_kv_heads, head_dim, flat)
+    return Plan(handle, R, num_q_heads, num_kv_heads, head_dim, flat, num_blocks)
 
 
 def _decode(fn_name: str, q, k_cache, v_cache, plan: "Plan", out, lse, scale, stream) -> None:
     lib = load_library()
     if scale is None:
         scale = 1.0 / math.sqrt(plan.head_dim)
-    for t, name in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (out, "out")):
-        if not t.is_cuda or str(t.dtype) != "torch.bfloat16" or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
-    if lse is not None and (str(lse.dtype) != "torch.float32" or not lse.is_contiguous()):
-        raise ValueError("lse must be a contiguous float32 CUDA tensor")
+    qshape = (plan.num_requests, plan.num_q_heads, plan.head_dim)
+    _check_bf16(q, "q", qshape)
+    _check_bf16(out, "out", qshape)
+    _check_caches(k_cache, v_cache, plan.num_blocks, plan.num_kv_heads, plan.head_dim)
+    _check_lse(lse, plan.num_requests, plan.num_q_heads)
     rc = getattr(lib, fn_name)(_ptr(q), _ptr(k_cache), _ptr(v_cache), plan.handle, _ptr(out),
                                _ptr(lse), float(scale), _stream_handle(stream))
     _check(rc, fn_name)
@@ -218,18 +248,22 @@ def fca_paged_decode_static(q, k_cache, v_cache, block_tables, seq_lens, num_blo
     CUDA tensor of one element (zeroed by the caller) or None.  Calls on one
     device must be ordered: they share the array."""
     lib = load_library()
-    for t, name in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (out, "out")):
-        if not t.is_cuda or str(t.dtype) != "torch.bfloat16" or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
-    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens")):
-        if not t.is_cuda or str(t.dtype) != "torch.int32" or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
-    if lse is not None and (str(lse.dtype) != "torch.float32" or not lse.is_contiguous()):
-        raise ValueError("lse must be a contiguous float32 CUDA tensor")
-    if dev_status is not None and (str(dev_status.dtype) != "torch.int32" or dev_status.numel() < 1):
-        raise ValueError("dev_status must be an int32 CUDA tensor of at least one element")
+    _check_bf16(q, "q")
+    if q.dim() != 3:
+        raise ValueError(f"q must be [R, Hq, D], not {tuple(q.shape)}")
     R, Hq, D = q.shape
+    _check_bf16(out, "out", q.shape)
+    if k_cache.dim() != 4:
+        raise ValueError(f"k_cache must be [num_blocks, 16, Hkv, D], not {tuple(k_cache.shape)}")
     Hkv = k_cache.shape[2]
+    _check_caches(k_cache, v_cache, num_blocks, Hkv, D)
+    _check_tables(block_tables, seq_lens)
+    if block_tables.shape[0] != R:
+        raise ValueError(f"block_tables must have {R} rows (one per request of q)")
+    _check_lse(lse, R, Hq)
+    if dev_status is not None and (not dev_status.is_cuda or str(dev_status.dtype) != "torch.int32"
+                                   or dev_status.numel() < 1):
+        raise ValueError("dev_status must be an int32 CUDA tensor of at least one element")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     rc = lib.fca_paged_decode_static(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
@@ -239,9 +273,15 @@ def fca_paged_decode_static(q, k_cache, v_cache, block_tables, seq_lens, num_blo
     _check(rc, "fca_paged_decode_static")
 
 
+def _check_pass_inputs(q, k_cache, v_cache, plan: "Plan") -> None:
+    _check_bf16(q, "q", (plan.num_requests, plan.num_q_heads, plan.head_dim))
+    _check_caches(k_cache, v_cache, plan.num_blocks, plan.num_kv_heads, plan.head_dim)
+
+
 def fca_prefix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) -> None:
     """Grouped pass over shared prefix blocks only (writes the plan's partials)."""
     scale = 1.0 / math.sqrt(plan.head_dim) if scale is None else scale
+    _check_pass_inputs(q, k_cache, v_cache, plan)
     _check(load_library().fca_prefix_pass(_ptr(q), _ptr(k_cache), _ptr(v_cache), plan.handle,
                                           float(scale), _stream_handle(stream)), "fca_prefix_pass")
 
@@ -249,12 +289,15 @@ def fca_prefix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) 
 def fca_suffix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) -> None:
     """Per-request pass over own blocks only (writes the plan's partials)."""
     scale = 1.0 / math.sqrt(plan.head_dim) if scale is None else scale
+    _check_pass_inputs(q, k_cache, v_cache, plan)
     _check(load_library().fca_suffix_pass(_ptr(q), _ptr(k_cache), _ptr(v_cache), plan.handle,
                                           float(scale), _stream_handle(stream)), "fca_suffix_pass")
 
 
 def fca_merge_pass(plan: "Plan", out, lse=None, stream=None) -> None:
     """Log-sum-exp merge of the plan's partials into out (and lse)."""
+    _check_bf16(out, "out", (plan.num_requests, plan.num_q_heads, plan.head_dim))
+    _check_lse(lse, plan.num_requests, plan.num_q_heads)
     _check(load_library().fca_merge_pass(plan.handle, _ptr(out), _ptr(lse), _stream_handle(stream)),
            "fca_merge_pass")
 
@@ -322,10 +365,12 @@ def fca_plan_destroy(plan: "Plan") -> None:
 class Plan:
     """Owner of an fca_plan_t handle."""
 
-    def __init__(self, handle: ctypes.c_void_p, R: int, Hq: int, Hkv: int, D: int, flat: bool):
+    def __init__(self, handle: ctypes.c_void_p, R: int, Hq: int, Hkv: int, D: int, flat: bool,
+                 num_blocks: int):
         self.handle = handle
         self.num_requests, self.num_q_heads, self.num_kv_heads, self.head_dim = R, Hq, Hkv, D
         self.flat = flat
+        self.num_blocks = num_blocks
 
     def stats(self) -> dict:
         return fca_plan_get_stats(self)
@@ -333,9 +378,7 @@ class Plan:
     def update(self, block_tables, seq_lens, stream=None) -> None:
         """Next decode step of the same batch (fca_plan_update): new lengths
         and grown tables over this plan's forest."""
-        for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens")):
-            if not t.is_cuda or str(t.dtype) != "torch.int32" or not t.is_contiguous():
-                raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+        _check_tables(block_tables, seq_lens)
         R, mb = block_tables.shape
         _check(load_library().fca_plan_update(self.handle, _ptr(block_tables), mb, _ptr(seq_lens), R,
                                               _stream_handle(stream)), "fca_plan_update")
