@@ -77,9 +77,11 @@ typedef struct fca_plan_opts {
                                   blocks -- the block reads sharing it saves -- reaches
                                   this; otherwise it is folded like a short group
                                   (>= 0; default 32, 0 = use every shared prefix).  The
-                                  automatic activation of "Core Mechanism": groups too
-                                  small to pay for their own grouped-pass work are
-                                  read by their members' own passes instead. */
+                                  reading here of FCA's automatic activation ("ZoRRo
+                                  Inference & Forest Cascade Attention", "How It
+                                  Works"): groups too small to pay for their own
+                                  grouped-pass work are read by their members' own
+                                  passes instead. */
 } fca_plan_opts;
 
 /* Build a plan with no groups: every request reads its whole table in its own
