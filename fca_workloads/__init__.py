@@ -43,6 +43,7 @@ Named configurations (one layer's decode step each):
 from __future__ import annotations
 
 import ctypes
+import bisect
 import dataclasses
 import math
 import os
@@ -152,14 +153,19 @@ def layout(requests, rng: np.random.Generator, block_size: int = BLOCK_SIZE,
 
     ``requests[r]`` is a list of ``(key, n_tokens)``; ``key`` names a shared
     prompt segment (requests whose leading keys agree share those tokens) and
-    ``None`` marks the request's own tokens.  Shared keys must come first.
-    Returns (block_tables, seq_lens, num_blocks, tail_copies) where
-    ``tail_copies`` lists (dst_block, src_block, n_tokens): private blocks whose
-    first tokens copy a shared prompt's tail.
+    ``None`` marks the request's own tokens.  Shared keys must come first, and
+    a key names its whole path (the same key never follows two different
+    paths).
+    Returns (block_tables, seq_lens, num_blocks, copies) where ``copies`` is a
+    list of (dst_block, dst_slot, src_block, src_slot): prompt tokens that sit
+    in more than one physical block (a block that holds the end of one prompt
+    segment and the start of the next, or a private block that holds a
+    prompt's partial tail) take the content of the token's first copy, as
+    copy-on-write leaves them.  A source slot is never a destination.
     """
     key_to_id = {}
-    tail_src = {}
-    tail_copies = []
+    first_slot = {}     # (segment key, offset in the segment) -> (block, slot) of its first copy
+    copies = []
     tables, lens = [], []
     next_id = 0
     for segs in requests:
@@ -175,22 +181,34 @@ def layout(requests, rng: np.random.Generator, block_size: int = BLOCK_SIZE,
             shared += int(n)
         row = []
         for j in range((L + block_size - 1) // block_size):
-            end = (j + 1) * block_size
+            lo, end = j * block_size, (j + 1) * block_size
             if end <= shared:
                 keys = tuple(k for k, s in zip(path, starts) if s < end)
                 bid = key_to_id.get((keys, j))
-                if bid is None:
+                new = bid is None
+                if new:
                     bid = key_to_id[(keys, j)] = next_id
                     next_id += 1
             else:
                 bid = next_id
                 next_id += 1
-                if j * block_size < shared:   # private copy of a shared tail
-                    tk = (tuple(path), j)
-                    if tk in tail_src:
-                        tail_copies.append((bid, tail_src[tk], shared - j * block_size))
-                    else:
-                        tail_src[tk] = bid
+                new = True
+            hi = min(end, shared)
+            if new and lo < hi:
+                seg_lo = bisect.bisect_right(starts, lo) - 1
+                seg_hi = bisect.bisect_right(starts, hi - 1) - 1
+                # only a block that spans a segment boundary, or holds a
+                # prompt's tail next to private tokens, can hold prompt tokens
+                # that another physical block also holds
+                if seg_lo != seg_hi or end > shared:
+                    for t in range(lo, hi):
+                        sg = bisect.bisect_right(starts, t) - 1
+                        ck = (path[sg], t - starts[sg])
+                        src = first_slot.get(ck)
+                        if src is None:
+                            first_slot[ck] = (bid, t - lo)
+                        else:
+                            copies.append((bid, t - lo, src[0], src[1]))
             row.append(bid)
         tables.append(row)
         lens.append(L)
@@ -202,15 +220,15 @@ def layout(requests, rng: np.random.Generator, block_size: int = BLOCK_SIZE,
     bt = rng.integers(0, num_blocks, size=(len(tables), mb), dtype=np.int32)  # padding
     for r, row in enumerate(tables):
         bt[r, :len(row)] = perm[np.asarray(row, dtype=np.int64)]
-    tail_copies = [(int(perm[d]), int(perm[s]), n) for d, s, n in tail_copies]
-    return bt, np.asarray(lens, np.int32), num_blocks, tail_copies
+    copies = [(int(perm[d]), so, int(perm[sb]), ss) for d, so, sb, ss in copies]
+    return bt, np.asarray(lens, np.int32), num_blocks, copies
 
 
 def fill(name: str, requests, Hq: int, Hkv: int, D: int, seed: int,
          rng: np.random.Generator, block_size: int = BLOCK_SIZE, k_boost_frac: float = 0.0,
          k_boost: float = 3.0, poison_padding: bool = False, description: str = "") -> Workload:
     """Lay out ``requests`` and draw Q, K and V."""
-    bt, sl, nb, tails = layout(requests, rng, block_size)
+    bt, sl, nb, copies = layout(requests, rng, block_size)
     R = len(requests)
     slots = nb * block_size
     row_factor = None
@@ -229,9 +247,10 @@ def fill(name: str, requests, Hq: int, Hkv: int, D: int, seed: int,
     kv_shape = (nb, block_size, Hkv, D)
     k = normal_bf16(kv_shape, seed, 1, row_factor, Hkv * D)
     v = normal_bf16(kv_shape, seed, 2)
-    for dst, src, n in tails:
-        k[dst, :n] = k[src, :n]
-        v[dst, :n] = v[src, :n]
+    if copies:
+        c = np.asarray(copies, np.int64)
+        k[c[:, 0], c[:, 1]] = k[c[:, 2], c[:, 3]]
+        v[c[:, 0], c[:, 1]] = v[c[:, 2], c[:, 3]]
     if poison_padding:
         # slots past every referencing request's length hold NaN: never read
         used = np.zeros(slots, bool)
