@@ -181,6 +181,7 @@ int oracle_paged_attention(const uint16_t *q, const uint16_t *k_cache,
         double *kd = (double *)malloc(sizeof(double) * (size_t)L * D);
         double *vd = (double *)malloc(sizeof(double) * (size_t)L * D);
         if (!qd || !kd || !vd) {
+#pragma omp atomic write
             status = ORACLE_ERR_NOMEM;
             free(qd); free(kd); free(vd);
             continue;
@@ -196,7 +197,10 @@ int oracle_paged_attention(const uint16_t *q, const uint16_t *k_cache,
             }
         }
         int rc = oracle_attend(qd, kd, vd, L, D, scale, out + i * D, lse + i);
-        if (rc != ORACLE_OK) status = rc;
+        if (rc != ORACLE_OK) {
+#pragma omp atomic write
+            status = rc;
+        }
         free(qd); free(kd); free(vd);
     }
     return status;
