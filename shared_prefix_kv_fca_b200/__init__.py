@@ -349,6 +349,15 @@ def fca_check_device_status(plan: "Plan", stream=None) -> int:
     return int(code.value)
 
 
+def fca_plan_update(plan: "Plan", block_tables, seq_lens, stream=None) -> None:
+    """The plan for the next decode step of the same batch: new lengths and
+    grown tables over the plan's forest (the C call of the same name)."""
+    _check_tables(block_tables, seq_lens)
+    R, mb = block_tables.shape
+    _check(load_library().fca_plan_update(plan.handle, _ptr(block_tables), mb, _ptr(seq_lens), R,
+                                          _stream_handle(stream)), "fca_plan_update")
+
+
 def fca_selftest_wait_timeout(stream=None) -> int:
     """Run the kernel whose bounded wait is made to run out; return the device
     error word it recorded (bit 1: the wait gave up after its 1 s bound)."""
@@ -378,10 +387,7 @@ class Plan:
     def update(self, block_tables, seq_lens, stream=None) -> None:
         """Next decode step of the same batch (fca_plan_update): new lengths
         and grown tables over this plan's forest."""
-        _check_tables(block_tables, seq_lens)
-        R, mb = block_tables.shape
-        _check(load_library().fca_plan_update(self.handle, _ptr(block_tables), mb, _ptr(seq_lens), R,
-                                              _stream_handle(stream)), "fca_plan_update")
+        fca_plan_update(self, block_tables, seq_lens, stream)
 
     def export(self) -> dict:
         return fca_plan_export(self)

@@ -99,3 +99,9 @@ def test_selftest_binding_without_a_device(lib):
     with pytest.raises(fca.FcaError) as ei:
         fca.fca_selftest_wait_timeout(stream=0)
     assert ei.value.status == 4
+
+
+def test_binding_has_every_entry_point_under_its_c_name():
+    # the Python layer is a thin binding: one function per C entry point, same name
+    missing = [n for n in declared_functions() if not callable(getattr(fca, n, None))]
+    assert not missing, missing

@@ -137,6 +137,11 @@ def test_tables_must_agree_with_each_other(lib):
     # a request fewer in both is the library's to refuse (it knows the plan's size)
     plan.update(t.bt[:-1], t.sl[:-1], stream=0)
     assert lib.calls.count("fca_plan_update") == 1
+    # the module-level call of the C name is the same call
+    fca.fca_plan_update(plan, t.bt, t.sl, stream=0)
+    with pytest.raises(ValueError):
+        fca.fca_plan_update(plan, t.bt, t.sl.to(torch.int64), stream=0)
+    assert lib.calls.count("fca_plan_update") == 2
 
 
 def test_static_decode_checks_its_tensors(lib):
