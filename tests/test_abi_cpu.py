@@ -6,6 +6,7 @@ No GPU needed: only calls that return before touching the device are made
 import ctypes
 import os
 import re
+import shutil
 import subprocess
 
 import pytest
@@ -105,3 +106,34 @@ def test_binding_has_every_entry_point_under_its_c_name():
     # the Python layer is a thin binding: one function per C entry point, same name
     missing = [n for n in declared_functions() if not callable(getattr(fca, n, None))]
     assert not missing, missing
+
+
+def test_header_is_plain_c(tmp_path):
+    # the public header compiles on its own as pedantic C99 and as C++
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    header = os.path.join(ROOT, "include", "fca.h")
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                           "-x", "c", header])
+    gxx = shutil.which("g++")
+    if gxx is not None:
+        subprocess.check_call([gxx, "-std=c++11", "-Wall", "-Werror", "-fsyntax-only", "-x", "c++", header])
+
+
+def test_c_client_links_and_runs(tmp_path, lib):
+    # a C99 program linked against the library calls it through the header alone
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(fca.library_path())
+    exe = str(tmp_path / "abi_c_client")
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Werror", "-I" + os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "abi_c_client.c"), "-L" + libdir, "-lfca_b200",
+                           "-Wl,-rpath," + libdir, "-o", exe])
+    out = subprocess.check_output([exe]).decode().strip()
+    version, msg, s_plan, s_dim, no_plan, s_upd, s_self, s_destroy, mgs, msv, word = out.split("|")
+    assert version == fca.fca_version()
+    assert msg == "block id out of range"
+    assert (s_plan, s_dim, no_plan, s_upd, s_self, s_destroy) == ("1", "3", "1", "1", "1", "0")
+    assert (mgs, msv, word) == ("2", "32", "-1")
