@@ -96,7 +96,7 @@ def test_selftest_binding_without_a_device(lib):
     # (no device); on a GPU machine the gpu-marked test runs the kernel itself
     import torch
     if torch.cuda.is_available():
-        pytest.skip("a device is present: tests/test_zzz_failure_detection.py covers the call")
+        pytest.skip("a device is present: tests/test_zy_failure_detection.py covers the call")
     with pytest.raises(fca.FcaError) as ei:
         fca.fca_selftest_wait_timeout(stream=0)
     assert ei.value.status == 4
