@@ -17,6 +17,7 @@ a log-sum-exp weighted merge; equal to standard attention.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -131,11 +132,42 @@ def _ptr(t) -> Optional[int]:
     return int(t.data_ptr())
 
 
-def _stream_handle(stream) -> Optional[int]:
+def _stream_handle(stream, device: Optional[int] = None) -> Optional[int]:
+    """The cudaStream_t of `stream`; None means torch's current stream of
+    `device` (of the current device when that is None too)."""
     if stream is None:
         import torch
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _one_device(*named) -> int:
+    """Index of the CUDA device that every given (name, tensor) pair is on.
+
+    The C entry points take raw pointers and run on one device (the plan's,
+    or the current one); a buffer on another device would be dereferenced
+    there, which is a fault, not an error code.  So a mismatch is refused
+    here, before anything reaches the library."""
+    idx, first = None, None
+    for name, t in named:
+        if t is None:
+            continue
+        i = t.device.index
+        if idx is None:
+            idx, first = i, name
+        elif i != idx:
+            raise ValueError(f"{name} is on cuda:{i} but {first} is on cuda:{idx}: "
+                             "every buffer of a call must be on one device")
+    return idx
+
+
+def _on_device(idx: Optional[int]):
+    """Context that makes CUDA device `idx` current for the call (no change
+    when no tensor named a device)."""
+    if idx is None:
+        return contextlib.nullcontext()
+    import torch
+    return torch.cuda.device(idx)
 
 
 def _check_tables(block_tables, seq_lens) -> None:
@@ -203,15 +235,17 @@ def fca_plan(block_tables, seq_lens, num_blocks: int, num_q_heads: int, num_kv_h
     folded (0 keeps every shared prefix)."""
     lib = load_library()
     _check_tables(block_tables, seq_lens)
+    dev = _one_device(("block_tables", block_tables), ("seq_lens", seq_lens))
     R, mb = block_tables.shape
     o = fca_plan_opts(min_group_size, min_shared_blocks, split_tokens, FCA_PLAN_FLAT if flat else 0,
                       min_saved_blocks)
     handle = ctypes.c_void_p()
-    rc = lib.fca_plan(_ptr(block_tables), mb, _ptr(seq_lens), R, block_size, num_blocks, num_q_heads,
-                      num_kv_heads, head_dim, ctypes.byref(o), ctypes.byref(handle),
-                      _stream_handle(stream))
+    with _on_device(dev):       # the plan belongs to the device current when it is built
+        rc = lib.fca_plan(_ptr(block_tables), mb, _ptr(seq_lens), R, block_size, num_blocks, num_q_heads,
+                          num_kv_heads, head_dim, ctypes.byref(o), ctypes.byref(handle),
+                          _stream_handle(stream, dev))
     _check(rc, "fca_plan")
-    return Plan(handle, R, num_q_heads, num_kv_heads, head_dim, flat, num_blocks)
+    return Plan(handle, R, num_q_heads, num_kv_heads, head_dim, flat, num_blocks, dev)
 
 
 def _decode(fn_name: str, q, k_cache, v_cache, plan: "Plan", out, lse, scale, stream) -> None:
@@ -223,9 +257,19 @@ def _decode(fn_name: str, q, k_cache, v_cache, plan: "Plan", out, lse, scale, st
     _check_bf16(out, "out", qshape)
     _check_caches(k_cache, v_cache, plan.num_blocks, plan.num_kv_heads, plan.head_dim)
     _check_lse(lse, plan.num_requests, plan.num_q_heads)
+    _plan_device(plan, ("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("out", out), ("lse", lse))
     rc = getattr(lib, fn_name)(_ptr(q), _ptr(k_cache), _ptr(v_cache), plan.handle, _ptr(out),
-                               _ptr(lse), float(scale), _stream_handle(stream))
+                               _ptr(lse), float(scale), _stream_handle(stream, plan.device))
     _check(rc, fn_name)
+
+
+def _plan_device(plan: "Plan", *named) -> None:
+    """Every buffer of a call that takes a plan must be on the plan's device
+    (the library makes that device current for the call)."""
+    idx = _one_device(*named)
+    if idx is not None and plan.device is not None and idx != plan.device:
+        name = next(n for n, t in named if t is not None)
+        raise ValueError(f"{name} is on cuda:{idx} but the plan belongs to cuda:{plan.device}")
 
 
 def fca_decode(q, k_cache, v_cache, plan: "Plan", out, lse=None, scale=None, stream=None) -> None:
@@ -264,18 +308,22 @@ def fca_paged_decode_static(q, k_cache, v_cache, block_tables, seq_lens, num_blo
     if dev_status is not None and (not dev_status.is_cuda or str(dev_status.dtype) != "torch.int32"
                                    or dev_status.numel() < 1):
         raise ValueError("dev_status must be an int32 CUDA tensor of at least one element")
+    dev = _one_device(("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("block_tables", block_tables),
+                      ("seq_lens", seq_lens), ("out", out), ("lse", lse), ("dev_status", dev_status))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    rc = lib.fca_paged_decode_static(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
-                                     block_tables.shape[1], _ptr(seq_lens), R, num_blocks, Hq, Hkv, D,
-                                     _ptr(out), _ptr(lse), float(scale), _ptr(dev_status),
-                                     _stream_handle(stream))
+    with _on_device(dev):       # the call runs on (and finds its array on) the current device
+        rc = lib.fca_paged_decode_static(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                         block_tables.shape[1], _ptr(seq_lens), R, num_blocks, Hq, Hkv, D,
+                                         _ptr(out), _ptr(lse), float(scale), _ptr(dev_status),
+                                         _stream_handle(stream, dev))
     _check(rc, "fca_paged_decode_static")
 
 
 def _check_pass_inputs(q, k_cache, v_cache, plan: "Plan") -> None:
     _check_bf16(q, "q", (plan.num_requests, plan.num_q_heads, plan.head_dim))
     _check_caches(k_cache, v_cache, plan.num_blocks, plan.num_kv_heads, plan.head_dim)
+    _plan_device(plan, ("q", q), ("k_cache", k_cache), ("v_cache", v_cache))
 
 
 def fca_prefix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) -> None:
@@ -283,7 +331,7 @@ def fca_prefix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) 
     scale = 1.0 / math.sqrt(plan.head_dim) if scale is None else scale
     _check_pass_inputs(q, k_cache, v_cache, plan)
     _check(load_library().fca_prefix_pass(_ptr(q), _ptr(k_cache), _ptr(v_cache), plan.handle,
-                                          float(scale), _stream_handle(stream)), "fca_prefix_pass")
+                                          float(scale), _stream_handle(stream, plan.device)), "fca_prefix_pass")
 
 
 def fca_suffix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) -> None:
@@ -291,14 +339,15 @@ def fca_suffix_pass(q, k_cache, v_cache, plan: "Plan", scale=None, stream=None) 
     scale = 1.0 / math.sqrt(plan.head_dim) if scale is None else scale
     _check_pass_inputs(q, k_cache, v_cache, plan)
     _check(load_library().fca_suffix_pass(_ptr(q), _ptr(k_cache), _ptr(v_cache), plan.handle,
-                                          float(scale), _stream_handle(stream)), "fca_suffix_pass")
+                                          float(scale), _stream_handle(stream, plan.device)), "fca_suffix_pass")
 
 
 def fca_merge_pass(plan: "Plan", out, lse=None, stream=None) -> None:
     """Log-sum-exp merge of the plan's partials into out (and lse)."""
     _check_bf16(out, "out", (plan.num_requests, plan.num_q_heads, plan.head_dim))
     _check_lse(lse, plan.num_requests, plan.num_q_heads)
-    _check(load_library().fca_merge_pass(plan.handle, _ptr(out), _ptr(lse), _stream_handle(stream)),
+    _plan_device(plan, ("out", out), ("lse", lse))
+    _check(load_library().fca_merge_pass(plan.handle, _ptr(out), _ptr(lse), _stream_handle(stream, plan.device)),
            "fca_merge_pass")
 
 
@@ -340,7 +389,7 @@ def fca_plan_export(plan: "Plan") -> dict:
 def fca_check_device_status(plan: "Plan", stream=None) -> int:
     """Raw device error word (0 = fine); raises FcaError when it is set."""
     code = ctypes.c_int32()
-    rc = load_library().fca_check_device_status(plan.handle, _stream_handle(stream),
+    rc = load_library().fca_check_device_status(plan.handle, _stream_handle(stream, plan.device),
                                                 ctypes.byref(code))
     if rc not in (0, 6):
         _check(rc, "fca_check_device_status")
@@ -353,9 +402,10 @@ def fca_plan_update(plan: "Plan", block_tables, seq_lens, stream=None) -> None:
     """The plan for the next decode step of the same batch: new lengths and
     grown tables over the plan's forest (the C call of the same name)."""
     _check_tables(block_tables, seq_lens)
+    _plan_device(plan, ("block_tables", block_tables), ("seq_lens", seq_lens))
     R, mb = block_tables.shape
     _check(load_library().fca_plan_update(plan.handle, _ptr(block_tables), mb, _ptr(seq_lens), R,
-                                          _stream_handle(stream)), "fca_plan_update")
+                                          _stream_handle(stream, plan.device)), "fca_plan_update")
 
 
 def fca_selftest_wait_timeout(stream=None) -> int:
@@ -375,11 +425,12 @@ class Plan:
     """Owner of an fca_plan_t handle."""
 
     def __init__(self, handle: ctypes.c_void_p, R: int, Hq: int, Hkv: int, D: int, flat: bool,
-                 num_blocks: int):
+                 num_blocks: int, device: Optional[int] = None):
         self.handle = handle
         self.num_requests, self.num_q_heads, self.num_kv_heads, self.head_dim = R, Hq, Hkv, D
         self.flat = flat
         self.num_blocks = num_blocks
+        self.device = device        # CUDA device index the plan belongs to
 
     def stats(self) -> dict:
         return fca_plan_get_stats(self)

@@ -156,3 +156,49 @@ def test_static_decode_checks_its_tensors(lib):
             fca.fca_paged_decode_static(a["q"], a["k"], a["v"], a["bt"], a["sl"], NB, a["out"], a["lse"], 0.125,
                                         dev_status=a["status"], stream=0)
     assert "fca_paged_decode_static" not in lib.calls
+
+
+class OnDevice:
+    """A CPU tensor that reports itself as living on CUDA device `idx`."""
+
+    def __init__(self, t, idx):
+        self._t = t
+        self.device = torch.device("cuda", idx)
+
+    def __getattr__(self, name):
+        return getattr(self._t, name)
+
+
+def test_buffers_on_another_device_are_refused(lib):
+    # a pointer on another device would be dereferenced on the device the call
+    # runs on: refused before anything reaches the library
+    t = tensors()
+    on = lambda x, i: OnDevice(x, i)          # noqa: E731
+    with pytest.raises(ValueError, match="one device"):
+        fca.fca_plan(on(t.bt, 0), on(t.sl, 1), NB, HQ, HKV, D, stream=0)
+    assert lib.calls == []
+    with pytest.raises(ValueError, match="one device"):
+        fca.fca_paged_decode_static(on(t.q, 0), on(t.k, 0), on(t.v, 0), on(t.bt, 0), on(t.sl, 0), NB,
+                                    on(t.out, 1), on(t.lse, 0), 0.125, stream=0)
+    with pytest.raises(ValueError, match="one device"):
+        fca.fca_paged_decode_static(on(t.q, 0), on(t.k, 0), on(t.v, 0), on(t.bt, 0), on(t.sl, 0), NB,
+                                    on(t.out, 0), on(t.lse, 0), 0.125,
+                                    dev_status=on(torch.zeros(1, dtype=torch.int32), 2), stream=0)
+    assert lib.calls == []
+    plan = make_plan(t)
+    plan.device = 0
+    q1, k1, v1, out1, lse1 = (on(x, 1) for x in (t.q, t.k, t.v, t.out, t.lse))
+    with pytest.raises(ValueError, match="plan belongs to cuda:0"):
+        fca.fca_decode(q1, k1, v1, plan, out1, lse1, 0.125, stream=0)
+    with pytest.raises(ValueError, match="plan belongs to cuda:0"):
+        fca.fca_prefix_pass(q1, k1, v1, plan, 0.125, stream=0)
+    with pytest.raises(ValueError, match="plan belongs to cuda:0"):
+        fca.fca_merge_pass(plan, out1, lse1, stream=0)
+    with pytest.raises(ValueError, match="plan belongs to cuda:0"):
+        plan.update(on(t.bt, 1), on(t.sl, 1), stream=0)
+    with pytest.raises(ValueError, match="one device"):
+        fca.fca_decode(on(t.q, 0), on(t.k, 0), on(t.v, 1), plan, on(t.out, 0), on(t.lse, 0), 0.125, stream=0)
+    assert lib.calls == ["fca_plan"]
+    # all on the plan's device: passes through
+    fca.fca_decode(*(on(x, 0) for x in (t.q, t.k, t.v)), plan, on(t.out, 0), on(t.lse, 0), 0.125, stream=0)
+    assert lib.calls == ["fca_plan", "fca_decode"]
