@@ -272,9 +272,8 @@ fca_status fca_selftest_wait_timeout(void *stream, int32_t *out_word);
  * fca_paged_decode_static -- the flat paged decode of fca_flat_decode
  * (standard split-KV attention of every request over its whole block table,
  * then the log-sum-exp merge) in one call that allocates nothing.  This entry
- * has no counterpart in the method's description ("ZoRRo Inference & Forest
- * Cascade Attention"); it is for callers that cannot allocate device memory
- * at decode time: an engine whose device memory is all handed out by its own
+ * has no counterpart in the method's description; it is for callers that
+ * cannot allocate device memory at decode time: an engine whose device memory is all handed out by its own
  * pool, or code that must not call the CUDA allocator while it records a
  * stream.  It needs no plan; it does not share prefix blocks.
  *
@@ -285,7 +284,12 @@ fca_status fca_selftest_wait_timeout(void *stream, int32_t *out_word);
  * it issues one cudaMemsetAsync of 16 bytes and three kernels on `stream`.
  * The first call on a device looks the array's address up
  * (cudaGetSymbolAddress), which may load the library's kernels on that
- * device; make that first call before any stream capture.
+ * device; make that first call before any stream capture.  The address is
+ * kept for the life of the process: do not call this entry point on a device
+ * after cudaDeviceReset (or another release of its primary context) in the
+ * same process, since the array may then sit elsewhere.
+ * q, k_cache, v_cache, block_tables, seq_lens, out, lse and dev_status must
+ * all be on the current device.
  *
  * What must start at zero: the array's three work counters, which the call
  * zeroes itself on `stream` before its kernels; and *dev_status, which the
