@@ -417,6 +417,31 @@ def test_unique_kv_tokens_hand_count():
     assert oracle.unique_kv_tokens(bt, sl, 16, 10) == 48 + 5 + 12 + 16 + 11
 
 
+def test_unique_kv_tokens_shared_partial_block_counts_its_longest_use():
+    # physical block 5 is the partly filled second block of requests 0 and 1
+    # (4 and 10 valid tokens) and the full first block of request 2; block 3
+    # holds 2 tokens of request 2.  Each physical slot is read once, so block 5
+    # counts 16 tokens (its longest use), not 4 + 10 + 16.
+    bt = np.array([[7, 5], [7, 5], [5, 3]], np.int32)
+    sl = np.array([20, 26, 18], np.int32)
+    assert oracle.unique_kv_tokens(bt, sl, 16, 8) == 16 + 16 + 2
+    # without request 2, block 5's longest use is request 1's 10 tokens
+    assert oracle.unique_kv_tokens(bt[:2], sl[:2], 16, 8) == 16 + 10
+    # one request alone: every slot it reads
+    assert oracle.unique_kv_tokens(bt[:1], sl[:1], 16, 8) == 20
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_unique_kv_tokens_is_the_number_of_distinct_slots(seed):
+    # brute force: the set of (physical block, slot) pairs any request reads
+    w = fca_workloads.random_small(seed, max_requests=24)
+    slots = set()
+    for r in range(w.R):
+        for t in range(int(w.seq_lens[r])):
+            slots.add((int(w.block_tables[r, t // 16]), t % 16))
+    assert oracle.unique_kv_tokens(w.block_tables, w.seq_lens, 16, w.num_blocks) == len(slots)
+
+
 def test_kv_bytes_per_token_worked_example():
     with open(os.path.join(GOLDEN, "kv_bytes_llama3_8b.json")) as f:
         g = json.load(f)
