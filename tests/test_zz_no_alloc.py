@@ -5,7 +5,7 @@ of a plan's workspace.  The GPU tests call it twice in a row through the C
 ABI and compare each result with fca_flat_decode (the existing entry point
 running the same kernels from a plan) on the same inputs, within twice the
 oracle tolerance (each side is within the oracle tolerance of the exact
-result), and the small cases with the oracle itself.  The file is named to be
+result), and with the oracle itself.  The file is named to be
 collected last, so it also runs after every other test has used the device.
 """
 import ctypes
@@ -126,7 +126,7 @@ def test_static_matches_flat_decode_head_dim_64():
 
 @pytest.mark.gpu
 def test_static_matches_flat_decode_full_size():
-    _two_calls_match_flat(fca_workloads.make("llama8b"), check_oracle=False)
+    _two_calls_match_flat(fca_workloads.make("llama8b"), check_oracle=True)
 
 
 @pytest.mark.gpu
