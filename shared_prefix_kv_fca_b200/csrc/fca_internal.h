@@ -15,7 +15,7 @@ namespace fca {
 
 constexpr int kBlockSize = 16;        // tokens per paged block (the only size built)
 constexpr int kPrefixTileRows = 128;  // stacked query rows per tcgen05 tile (MMA M)
-constexpr int kStageTokens = 64;      // tokens per pipeline stage of the grouped pass
+constexpr int kStageTokens = 128;     // tokens per pipeline stage of the grouped pass
 constexpr int kMaxGqa = 16;           // query heads per KV head handled by the own pass
 constexpr int kMaxRequests = 16384;   // groups are sorted in one CTA's shared memory
 constexpr int kMaxRequestsFallback = 4096;  // all-pairs LCP path (see fca_plan.cu)
