@@ -65,7 +65,16 @@ def parse():
                     help="also time a multi-layer step: one plan, then this many layers' decodes")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0,
                     help="approximate CPU seconds of the oracle baseline sample")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the lighter measurement of the other configurations")
+    ap.add_argument("--per-config-steps", type=int, default=10,
+                    help="timed steps per configuration in per_config")
     return ap.parse_args()
+
+
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+PER_CONFIGS = ("tiny", "llama8b", "longctx", "forest", "mixed")
 
 
 def peaks():
@@ -75,6 +84,41 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peaks():
+    """(bf16 burst TFLOP/s, bf16 sustained TFLOP/s, 'measured' | 'fallback')."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
+
+
+def prefix_flops(suffix_start, block_size: int, Hq: int, D: int) -> int:
+    """Algorithmic flops of the grouped pass: every query head of a request
+    attends every token its groups cover once (Q.K^T and P.V, 2 x 2 D flops
+    per query row and key).  A request's groups cover tokens
+    [0, suffix_start x block_size)."""
+    import numpy as np
+    return int(np.asarray(suffix_start, dtype=np.int64).sum()) * block_size * Hq * 4 * D
+
+
+def prefix_roofline(prefix_bytes: int, flops: int, prefix_ms: float, hbm_gbs: float, tflops_burst: float,
+                    tflops_sustained: float, peak_kind: str, tensor_pipe_pct=None):
+    """The grouped pass timed alone on every SM: K/V bytes it streams (each
+    shared token once per group) and its algorithmic flops over its duration,
+    as fractions of the measured copy bandwidth and bf16 tensor peaks."""
+    if prefix_ms is None or prefix_ms <= 0 or prefix_bytes <= 0:
+        return None
+    gbs = prefix_bytes / (prefix_ms * 1e-3) / 1e9
+    tfs = flops / (prefix_ms * 1e-3) / 1e12
+    return {"kernel": "k_prefix", "us": prefix_ms * 1e3, "algorithmic_bytes": int(prefix_bytes),
+            "algorithmic_flops": int(flops), "achieved_gbs": gbs, "frac_hbm": gbs / hbm_gbs,
+            "achieved_tflops": tfs, "frac_tensor_burst": tfs / tflops_burst,
+            "frac_tensor_sustained": tfs / tflops_sustained, "tensor_pipe_pct": tensor_pipe_pct,
+            "peak_note": f"{peak_kind} hbm_gbs, bf16_tflops and bf16_tflops_sustained"}
 
 
 def workload_desc(w):
@@ -296,21 +340,100 @@ def reference_arm(args):
 
 # ------------------------------------------------------------------ FCA arm
 
-def traffic_record(dominant: str, workload: str):
-    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+def traffic_entry(kernel: str, workload: str):
+    """The committed ncu record of a kernel on a workload (profiles/traffic.json),
     or None when there is none for this kernel source and workload."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
-        ent = rec[dominant][workload]
-        src = os.path.join(ROOT, "shared_prefix_kv_fca_b200", "csrc", DOMINANT_SOURCES[dominant])
+        ent = rec[kernel][workload]
+        src = os.path.join(ROOT, "shared_prefix_kv_fca_b200", "csrc", DOMINANT_SOURCES[kernel])
         digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         if ent.get("source_sha256_16") != digest:
             return None
-        return float(ent["dram_bytes_per_launch"])
+        return ent
     except Exception:
         return None
+
+
+def traffic_record(dominant: str, workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+    or None when there is none for this kernel source and workload."""
+    ent = traffic_entry(dominant, workload)
+    try:
+        return float(ent["dram_bytes_per_launch"]) if ent else None
+    except Exception:
+        return None
+
+
+def measure_config(name, args, dev, rank, flush, red, peak, prefix_line):
+    """One configuration, lighter than the headline: whole fca_decode steps
+    (L2 flushed before each), the three passes alone on every SM, and the flat
+    paged decode of the same batch; every rank decodes its own batch."""
+    import torch
+    import fca_workloads
+    import shared_prefix_kv_fca_b200 as fca
+
+    w = fca_workloads.make(name, seed=rank)
+    q, k, v, bt, sl = w.torch_inputs(dev)
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(w.R, w.Hq, dtype=torch.float32, device=dev)
+    n, warm = args.per_config_steps, max(3, min(args.warmup, 5))
+
+    def steps(p, flat=False):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for i in range(warm + n):
+            flush.zero_()
+            if i >= warm:
+                ev[i - warm][0].record(stream)
+            (fca.fca_flat_decode if flat else fca.fca_decode)(q, k, v, p, out, lse, w.scale, stream)
+            if i >= warm:
+                ev[i - warm][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return red.max(statistics.mean(a.elapsed_time(b) for a, b in ev))
+
+    def passes(p):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+        for i in range(warm + n):
+            flush.zero_()
+            e = ev[i - warm] if i >= warm else None
+            if e: e[0].record(stream)
+            fca.fca_prefix_pass(q, k, v, p, w.scale, stream)
+            if e: e[1].record(stream)
+            fca.fca_suffix_pass(q, k, v, p, w.scale, stream)
+            if e: e[2].record(stream)
+            fca.fca_merge_pass(p, out, lse, stream)
+            if e: e[3].record(stream)
+        torch.cuda.synchronize(dev)
+        return {key: red.max(statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev))
+                for i, key in enumerate(("prefix", "suffix", "merge"))}
+
+    plan = fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, split_tokens=args.split)
+    st, exp = plan.stats(), plan.export()
+    step_ms = steps(plan)
+    pass_ms = passes(plan)
+    assert fca.fca_check_device_status(plan, stream) == 0
+    flat_ms = None
+    if not args.no_flat:
+        flat = fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, flat=True, split_tokens=args.split)
+        flat_ms = steps(flat, flat=True)
+        assert fca.fca_check_device_status(flat, stream) == 0
+        flat.close()
+    total = red.sum(st["unique_kv_bytes"])
+    gbs = total / (step_ms * 1e-3) / 1e9
+    res = {"us_per_step": step_ms * 1e3, "unique_kv_gbs": gbs, "pct_of_peak": 100.0 * gbs / (peak * red.world),
+           "flat_us_per_step": flat_ms * 1e3 if flat_ms else None,
+           "speedup_vs_flat": (flat_ms / step_ms) if flat_ms else None,
+           "passes_us": {key: val * 1e3 for key, val in pass_ms.items()},
+           "roofline_prefix": prefix_line(st, exp, w, pass_ms["prefix"], name),
+           "unique_kv_bytes_per_rank": st["unique_kv_bytes"], "groups": st["num_groups"],
+           "workload": workload_desc(w)}
+    plan.close()
+    del q, k, v, bt, sl, out, lse
+    torch.cuda.empty_cache()
+    return res
 
 
 def fca_arm(args):
@@ -350,6 +473,17 @@ def fca_arm(args):
     torch.cuda.synchronize(dev)
     plan_ms = (time.perf_counter() - t0) * 1e3
     st = plan.stats()
+    exp = plan.export()
+    # the same plan again, as a decode loop that plans every step would: the
+    # first plan above also pays for the process's first pool allocations
+    steady = []
+    for _ in range(10):
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, split_tokens=args.split).close()
+        torch.cuda.synchronize(dev)
+        steady.append((time.perf_counter() - t0) * 1e3)
+    plan_ms_steady = statistics.median(steady)
     flat_plan = None if args.no_flat else fca.fca_plan(bt, sl, w.num_blocks, w.Hq, w.Hkv, w.D, flat=True,
                                                        split_tokens=args.split)
 
@@ -465,22 +599,32 @@ def fca_arm(args):
         side = torch.cuda.Stream(dev)
         q_ready = torch.cuda.Event()
 
-        def e2e_step():
+        parts = []
+
+        def e2e_step(record=False):
             # the planner needs only the tables: q is uploaded on a side
             # stream meanwhile, and the decode waits for it
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            ev[0].record(stream)
             side.wait_stream(stream)
             with torch.cuda.stream(side):
                 q_d.copy_(q_h, non_blocking=True)
                 q_ready.record(side)
             bt_d.copy_(bt_h, non_blocking=True)
             sl_d.copy_(sl_h, non_blocking=True)
+            ev[1].record(stream)
             with fca.fca_plan(bt_d, sl_d, w.num_blocks, w.Hq, w.Hkv, w.D, split_tokens=args.split,
                               stream=stream) as p:
                 stream.wait_event(q_ready)
+                ev[2].record(stream)
                 fca.fca_decode(q_d, k, v, p, out, lse, w.scale, stream)
+                ev[3].record(stream)
                 out_h.copy_(out, non_blocking=True)
                 lse_h.copy_(lse, non_blocking=True)
+                ev[4].record(stream)
                 torch.cuda.synchronize(dev)
+            if record:
+                parts.append([ev[i].elapsed_time(ev[i + 1]) for i in range(4)])
 
         for _ in range(max(1, args.warmup)):
             flush.zero_()
@@ -492,11 +636,13 @@ def fca_arm(args):
             torch.cuda.synchronize(dev)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            e2e_step()
+            e2e_step(record=True)
             b.record(stream)
             b.synchronize()
             times.append(a.elapsed_time(b))
         e2e_ms = max_over_ranks(statistics.mean(times))
+        e2e_parts = {key: max_over_ranks(statistics.mean(p[i] for p in parts))
+                     for i, key in enumerate(("h2d_tables_ms", "plan_ms", "decode_ms", "d2h_ms"))}
 
         # the same step in a decode loop that keeps its plan: fca_plan_update
         # (the tables' shared entries unchanged) in place of a new plan
@@ -539,6 +685,7 @@ def fca_arm(args):
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "includes": "H2D of the block tables, fca_plan (one host sync) while q uploads on a "
                            "side stream, fca_decode, D2H of out and lse; the KV cache is resident state",
+               "parts": e2e_parts,
                "with_plan_update": {"value": sum_over_ranks(st["unique_kv_bytes"]) / (upd_ms * 1e-3) / 1e9,
                                     "ms_per_step": upd_ms,
                                     "includes": "the same, with fca_plan_update of a kept plan in place "
@@ -579,6 +726,7 @@ def fca_arm(args):
                  "includes": "fca_plan (one host sync) then one fca_decode per layer over distinct caches"}
 
     peak, peak_kind = peaks()
+    tf_burst, tf_sust, tf_kind = tensor_peaks()
 
     # dominant kernel and its roofline
     pass_ms = {key: max_over_ranks(fca_t[key]) for key in ("prefix", "suffix", "merge")}
@@ -588,6 +736,32 @@ def fca_arm(args):
                  "merge": st["num_partials"] * (w.D + 1) * 4 + w.R * w.Hq * (w.D * 2 + 4)}
     achieved = alg_bytes[dominant] / (pass_ms[dominant] * 1e-3) / 1e9
     traffic = traffic_record(dominant, args.config)
+
+    def prefix_line(stats, export, wk, prefix_ms, workload):
+        ent = traffic_entry("prefix", workload)
+        return prefix_roofline(stats["prefix_kv_bytes"], prefix_flops(export["suffix_start"], wk.block_size, wk.Hq, wk.D),
+                               prefix_ms if stats["prefix_items"] > 0 else None, peak, tf_burst, tf_sust,
+                               f"{peak_kind}/{tf_kind}", ent.get("tensor_pipe_pct") if ent else None)
+
+    roof_prefix = prefix_line(st, exp, w, pass_ms["prefix"], args.config)
+
+    # ---- the other configurations, lighter: whole steps, the passes alone, flat
+    per_config = None
+    if not args.no_per_config and args.prompts is None:
+        per_config = {"steps": args.per_config_steps, "warmup": max(3, min(args.warmup, 5)),
+                      "note": "L2 flushed before every step; the headline configuration's entry repeats its "
+                              "own measurement"}
+        for name in PER_CONFIGS:
+            if name == args.config:
+                per_config[name] = {"us_per_step": step_ms * 1e3, "unique_kv_gbs": value,
+                                    "pct_of_peak": 100.0 * value / (peak * world),
+                                    "flat_us_per_step": flat_ms * 1e3 if flat_ms else None,
+                                    "speedup_vs_flat": (flat_ms / step_ms) if flat_ms else None,
+                                    "passes_us": {key: val * 1e3 for key, val in pass_ms.items()},
+                                    "roofline_prefix": roof_prefix}
+                continue
+            per_config[name] = measure_config(name, args, dev, rank, flush, red, peak, prefix_line)
+
 
     line = None
     if rank == 0:
@@ -621,7 +795,7 @@ def fca_arm(args):
                        "unique_kv_bytes_per_rank": st["unique_kv_bytes"],
                        "flat_kv_bytes_per_rank": st["flat_kv_bytes"], "replicas": world},
             "pct_of_peak": 100.0 * value / (peak * world), "peak_gbs": peak, "peak_kind": peak_kind,
-            "plan_ms": plan_ms,
+            "plan_ms": plan_ms, "plan_ms_steady": plan_ms_steady,
             "warm_l2_us_per_step": warm_ms * 1e3,
             "passes_us": {key: val * 1e3 for key, val in pass_ms.items()},
             "serial_passes_us_per_step": serial_ms * 1e3,
@@ -631,6 +805,7 @@ def fca_arm(args):
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_bytes": alg_bytes[dominant],
                          "peak_note": f"{peak_kind} copy bandwidth (MEASURED_PEAKS hbm_gbs)"},
+            "roofline_prefix": roof_prefix, "per_config": per_config,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "multilayer": multi,
             "gpu_launches": n_launch * args.steps, "impl": "fca",
         }

@@ -92,3 +92,23 @@ def test_gpu_id_for(monkeypatch, vis, local, want):
     else:
         monkeypatch.setenv("CUDA_VISIBLE_DEVICES", vis)
     assert bench.gpu_id_for(local) == want
+
+
+def test_prefix_flops_counts_each_shared_token_once_per_query_head():
+    # two requests whose groups cover 3 and 1 blocks of 16 tokens; 8 query
+    # heads of head_dim 128: 4 x 128 flops per (query head, key)
+    assert bench.prefix_flops([3, 1], 16, 8, 128) == (3 + 1) * 16 * 8 * 4 * 128
+    assert bench.prefix_flops([0, 0], 16, 8, 128) == 0
+
+
+def test_prefix_roofline_fractions():
+    r = bench.prefix_roofline(prefix_bytes=2_000_000_000, flops=4_000_000_000_000, prefix_ms=1.0, hbm_gbs=4000.0,
+                              tflops_burst=8000.0, tflops_sustained=5000.0, peak_kind="measured",
+                              tensor_pipe_pct=12.5)
+    assert abs(r["achieved_gbs"] - 2000.0) < 1e-9 and abs(r["frac_hbm"] - 0.5) < 1e-12
+    assert abs(r["achieved_tflops"] - 4000.0) < 1e-9
+    assert abs(r["frac_tensor_burst"] - 0.5) < 1e-12 and abs(r["frac_tensor_sustained"] - 0.8) < 1e-12
+    assert r["tensor_pipe_pct"] == 12.5 and r["us"] == 1000.0
+    # no grouped pass (flat plan, or no group): no roofline
+    assert bench.prefix_roofline(0, 0, 1.0, 1.0, 1.0, 1.0, "x") is None
+    assert bench.prefix_roofline(10, 10, None, 1.0, 1.0, 1.0, "x") is None
