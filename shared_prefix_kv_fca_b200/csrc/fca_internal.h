@@ -49,6 +49,10 @@ constexpr double kSuffixGBsPerSM = 49.0;
 // the flat decode.
 constexpr int32_t kDefaultMinSavedBlocks = 32;
 
+// Group partials per request whose rows the planner records for the merge
+// (more take the chain walk).
+constexpr int kMergeRec = 8;
+
 // Shortest chunk the per-request pass splits a request's own tokens into.
 // Longer chunks mean fewer partial rows to write and merge; a sweep of 256,
 // 384 and 512 on the four large workloads favoured 512 (forest 204 -> 195 us
@@ -149,6 +153,9 @@ struct fca_plan_s {
     float* part_o = nullptr;         // [n_partials][D]
     float* part_lse = nullptr;       // [n_partials]
     int32_t* dev_status = nullptr;   // device error word
+    int32_t* m_ng = nullptr;         // [R] partials per KV head from r's groups
+    int2* m_rec = nullptr;           // [R][kMergeRec] where they are: row of (KV head h, query head i)
+                                     // = x + h y + i (chain order; unused when m_ng > kMergeRec)
 
     // side stream and events for running the two passes side by side
     cudaStream_t aux_stream = nullptr;

@@ -46,6 +46,8 @@ struct MergeArgs {
     const float* part_lse;
     __nv_bfloat16* out;
     float* lse;
+    const int32_t* m_ng;      // null: walk the chain
+    const int2* m_rec;
 };
 
 namespace {
@@ -122,11 +124,28 @@ __global__ void __launch_bounds__(256, 3) k_merge(MergeArgs a) {
 
     if (active) {
         // ---- the request's partials: chain entries (one lane each), then its own chunks
-        const int32_t c0 = a.chain_off[r], depth = a.chain_off[r + 1] - c0;
         const int32_t nsc = a.s_nch[r], spart = a.s_part[r];
+        // The planner's record of the group partials (one entry each, read
+        // with the request's own counts, no dependent loads) when it holds
+        // them all; else the chain walk.
+        const int32_t ng = a.m_ng ? a.m_ng[r] : kMergeRec + 1;
+        // (read whatever the count is, so that it does not wait for the count)
+        const int2 rec = (a.m_rec && lane < kMergeRec) ? a.m_rec[(int64_t)r * kMergeRec + lane] : make_int2(0, 0);
+        const bool recorded = ng <= kMergeRec;
+        const int32_t c0 = recorded ? 0 : a.chain_off[r];
+        const int32_t depth = recorded ? ng : a.chain_off[r + 1] - c0;
         const bool wide = depth < 32;   // warp-uniform: every entry fits one lane
         int32_t e_nch = 0, e_base = 0, e_step = 0;
-        if (wide) {
+        if (recorded) {
+            if (lane < depth) {
+                e_nch = 1;
+                e_base = rec.x + h * rec.y + gq0;
+            } else if (lane == depth) {
+                e_nch = nsc;
+                e_base = spart + h * nsc * a.G + gq0;
+                e_step = a.G;
+            }
+        } else if (wide) {
             // entry e < depth: group chain[e]; row of (chunk k, slab) =
             //   g_part + ((h nch + k) nm + pos) G + gq0 = e_base + k * e_step
             // entry depth: own chunks, row = s_part + (h nsc + k) G + gq0
@@ -146,7 +165,7 @@ __global__ void __launch_bounds__(256, 3) k_merge(MergeArgs a) {
         int32_t n = nsc;
         if (wide) {
             n = __shfl_sync(kFull, e_end, depth);
-        } else {
+        } else {   // (never for a recorded request: depth <= kMergeRec)
             for (int32_t c = c0; c < c0 + depth; ++c) n += a.g_nch[a.chain_g[c]];
         }
 
@@ -305,6 +324,8 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, cudaStream_
     a.part_lse = P->part_lse;
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
+    a.m_ng = P->m_ng;
+    a.m_rec = P->m_rec;
     const int64_t units = (int64_t)P->R * P->Hkv * a.n_slabs;
     // Warps per unit: split a unit's partials over more warps only while the
     // whole grid stays under about 8 warps per SM and every warp still gets

@@ -779,6 +779,24 @@ __global__ void k_fill_suffix_items(int32_t R, const int32_t* seq_lens, const in
     }
 }
 
+// Per request, its group partials in chain order (the order the merge reads
+// them in): group g's chunk c holds member pos's G rows of KV head h at
+// g_part + ((h nch + c) nm + pos) G, i.e. x + h y with x = g_part + (c nm +
+// pos) G and y = nch nm G.  The first kMergeRec are recorded; m_ng counts all.
+__global__ void k_merge_records(int32_t R, int32_t G, const int32_t* chain_off, const int32_t* chain_g,
+                                const int32_t* chain_pos, const int32_t* g_nch, const int32_t* g_nm,
+                                const int32_t* g_part, int32_t* m_ng, int2* m_rec) {
+    for (int32_t r = blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x) {
+        int32_t k = 0;
+        for (int32_t c = chain_off[r]; c < chain_off[r + 1]; ++c) {
+            const int32_t g = chain_g[c], pos = chain_pos[c], nch = g_nch[g], nm = g_nm[g];
+            for (int32_t ch = 0; ch < nch; ++ch, ++k)
+                if (k < kMergeRec) m_rec[(int64_t)r * kMergeRec + k] = make_int2(g_part[g] + (ch * nm + pos) * G, nch * nm * G);
+        }
+        m_ng[r] = k;
+    }
+}
+
 // ------------------------------------------------------------ plan update
 
 // Thread (r, j): the entries of request r's table that its groups read (its
@@ -1025,6 +1043,8 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     pa.add(&P->s_chunk, R);
     pa.add(&P->g_wa, R);
     pa.add(&P->chain_off, R + 1);
+    pa.add(&P->m_ng, R);
+    pa.add(&P->m_rec, (size_t)R * kMergeRec);
     {
         void* base = nullptr;
         if (pa.commit(stream, &base) != cudaSuccess) {
@@ -1166,6 +1186,9 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
             R, P->seq_lens, P->suffix_start, P->s_nch, P->s_chunk, P->s_part, bin_cursor, G, Hkv, P->suffix_items);
         FCA_CK(cudaGetLastError());
     }
+    k_merge_records<<<grid_for(R, 128), 128, 0, stream>>>(R, G, P->chain_off, P->chain_g, P->chain_pos, P->g_nch,
+                                                          P->g_nm, P->g_part, P->m_ng, P->m_rec);
+    FCA_CK(cudaGetLastError());
     return FCA_OK;   // temporaries go back to the pool in stream order
 }
 
