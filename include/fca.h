@@ -166,14 +166,15 @@ fca_status fca_plan_update(fca_plan_t plan, const int32_t *block_tables, int32_t
  *   scale    multiplier of q.k (normally 1/sqrt(head_dim)); positive and finite,
  *            else FCA_ERR_INVALID_ARG.
  *
- * Asynchronous on `stream`.  When the plan has both grouped and per-request
- * work, the two passes run side by side on disjoint sets of SMs: the grouped
- * pass on a high-priority side stream that the plan creates on its first
- * decode (ordered after the work already queued on `stream` by an event),
- * the per-request pass on `stream`; the merge waits for both.  Uses the
- * plan's workspace, so decodes that share a plan must be ordered on one
- * stream.  A kernel that detects an internal error records it in the plan;
- * read it with fca_check_device_status.
+ * Asynchronous on `stream`, three kernels in order.  When the plan has both
+ * grouped and per-request work, the two passes share the SMs: the grouped
+ * pass takes its share, and the per-request pass (launched with programmatic
+ * stream serialization) starts on the other SMs as soon as the grouped pass
+ * runs, then takes over each SM the grouped pass gives up; it ends after the
+ * grouped pass, and the merge follows it.  Uses the plan's workspace, so
+ * decodes that share a plan must be ordered on one stream.  A kernel that
+ * detects an internal error records it in the plan; read it with
+ * fca_check_device_status.
  */
 fca_status fca_decode(const void *q, const void *k_cache, const void *v_cache, fca_plan_t plan,
                       void *out, float *lse, float scale, void *stream);

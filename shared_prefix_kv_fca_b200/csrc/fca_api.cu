@@ -15,8 +15,8 @@ fca_status plan_update(const int32_t* block_tables, const int32_t* seq_lens, cud
 cudaError_t launch_prefix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
                           float scale, int max_ctas, cudaStream_t stream);
 cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
-                          float scale, int max_ctas, cudaStream_t stream);
-cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, cudaStream_t stream);
+                          float scale, bool beside, cudaStream_t stream);
+cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_pass, cudaStream_t stream);
 
 namespace {
 thread_local cudaError_t g_last_error = cudaSuccess;
@@ -102,9 +102,6 @@ fca_status fca_plan_destroy(fca_plan_t plan) {
     cudaDeviceSynchronize();
     for (void* p : plan->dev_allocs) cudaFreeAsync(p, cudaStreamLegacy);
     cudaStreamSynchronize(cudaStreamLegacy);
-    if (plan->aux_stream) cudaStreamDestroy(plan->aux_stream);
-    if (plan->ev_fork) cudaEventDestroy(plan->ev_fork);
-    if (plan->ev_join) cudaEventDestroy(plan->ev_join);
     (void)cudaGetLastError();
     delete plan;
     return FCA_OK;
@@ -160,16 +157,22 @@ fca_status fca_plan_update(fca_plan_t plan, const int32_t* block_tables, int32_t
 }
 
 // SMs given to the grouped pass when it runs beside the per-request pass:
-// 0.9 of the share that would make both finish together at their measured
+// 1.15 x the share that would make both finish together at their measured
 // per-SM rates (kPrefixGBsPerSM, kSuffixGBsPerSM), the grouped pass's work
-// counted in tile-tokens.  A sweep of fixed splits on four workloads put this
-// next to the best split.  Each pass is launched on its own SMs: run on every
-// SM, the per-request pass shares SMs with the grouped one and slows it.
+// counted in tile-tokens, then trimmed to the fewest SMs that still take its
+// items in the same number of rounds.  The per-request pass starts on the
+// other SMs and takes over each SM the grouped pass gives up, so the grouped
+// pass must not be the last to finish: of 0.8, 0.9, 1.0 and 1.15, 1.15 gave
+// the fastest steps on the llama8b, longctx and mixed workloads (forest: the
+// same split from 0.9 up).
 static int prefix_share(const fca_plan_s* P, int sms) {
     const double tp = (double)P->hdr.prefix_tile_tok_sum / kPrefixGBsPerSM;
     const double ts = (double)P->hdr.suffix_tok_sum / kSuffixGBsPerSM;
-    const int n = (int)(0.9 * sms * tp / (tp + ts) + 0.5);
-    return std::max(1, std::min(sms - 1, n));
+    int n = (int)(1.15 * sms * tp / (tp + ts) + 0.5);
+    n = std::max(1, std::min(sms - 1, n));
+    const int items = P->hdr.n_prefix_items;
+    const int rounds = (items + n - 1) / n;
+    return std::max(1, std::min(n, (items + rounds - 1) / rounds));
 }
 
 static fca_status decode_impl(const void* q, const void* k_cache, const void* v_cache, fca_plan_t plan, void* out,
@@ -186,34 +189,21 @@ static fca_status decode_impl(const void* q, const void* k_cache, const void* v_
         !make_cache_map(&tv, v_cache, plan->num_blocks, plan->Hkv, plan->D))
         return FCA_ERR_CUDA;
     const bool grouped = !plan->flat && plan->hdr.n_prefix_items > 0;
-    if (grouped && plan->hdr.n_suffix_items > 0) {
-        // The two passes are independent: run them side by side on disjoint SMs.
-        if (!plan->aux_stream) {
-            // highest priority, so the grouped pass's CTAs are placed first
-            int lo = 0, hi = 0;
-            cudaDeviceGetStreamPriorityRange(&lo, &hi);
-            if (note_cuda(cudaStreamCreateWithPriority(&plan->aux_stream, cudaStreamNonBlocking, hi)) != cudaSuccess ||
-                note_cuda(cudaEventCreateWithFlags(&plan->ev_fork, cudaEventDisableTiming)) != cudaSuccess ||
-                note_cuda(cudaEventCreateWithFlags(&plan->ev_join, cudaEventDisableTiming)) != cudaSuccess)
-                return FCA_ERR_CUDA;
-        }
+    const bool own = plan->hdr.n_suffix_items > 0;
+    if (grouped) {
+        // The two passes are independent.  With both, they share the SMs: the
+        // grouped pass on its share, the per-request pass on the rest and then
+        // on every SM the grouped pass leaves (programmatic serialization: it
+        // starts once the grouped pass's CTAs all run, and ends after it).
         int dev = 0, sms = 148;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int np = prefix_share(plan, sms);
-        if (note_cuda(cudaEventRecord(plan->ev_fork, s)) != cudaSuccess ||
-            note_cuda(cudaStreamWaitEvent(plan->aux_stream, plan->ev_fork, 0)) != cudaSuccess ||
-            note_cuda(launch_prefix(plan, q, tk, tv, scale, np, plan->aux_stream)) != cudaSuccess ||
-            note_cuda(launch_suffix(plan, q, tk, tv, scale, sms - np, s)) != cudaSuccess ||
-            note_cuda(cudaEventRecord(plan->ev_join, plan->aux_stream)) != cudaSuccess ||
-            note_cuda(cudaStreamWaitEvent(s, plan->ev_join, 0)) != cudaSuccess)
-            return FCA_ERR_CUDA;
-    } else {
-        if (grouped && note_cuda(launch_prefix(plan, q, tk, tv, scale, 0, s)) != cudaSuccess)
-            return FCA_ERR_CUDA;
-        if (note_cuda(launch_suffix(plan, q, tk, tv, scale, 0, s)) != cudaSuccess) return FCA_ERR_CUDA;
+        const int np = own ? prefix_share(plan, sms) : 0;
+        if (note_cuda(launch_prefix(plan, q, tk, tv, scale, np, s)) != cudaSuccess) return FCA_ERR_CUDA;
     }
-    if (note_cuda(launch_merge(plan, out, lse, s)) != cudaSuccess) return FCA_ERR_CUDA;
+    if (own && note_cuda(launch_suffix(plan, q, tk, tv, scale, grouped, s)) != cudaSuccess) return FCA_ERR_CUDA;
+    // behind the per-request pass, which ends after the grouped one
+    if (note_cuda(launch_merge(plan, out, lse, own, s)) != cudaSuccess) return FCA_ERR_CUDA;
     return FCA_OK;
 }
 
@@ -238,7 +228,7 @@ static fca_status pass_impl(int pass, const void* q, const void* k_cache, const 
         return note_cuda(launch_prefix(plan, q, tk, tv, scale, 0, s)) == cudaSuccess ? FCA_OK
                                                                                                    : FCA_ERR_CUDA;
     }
-    return note_cuda(launch_suffix(plan, q, tk, tv, scale, 0, s)) == cudaSuccess ? FCA_OK : FCA_ERR_CUDA;
+    return note_cuda(launch_suffix(plan, q, tk, tv, scale, false, s)) == cudaSuccess ? FCA_OK : FCA_ERR_CUDA;
 }
 
 fca_status fca_prefix_pass(const void* q, const void* k_cache, const void* v_cache, fca_plan_t plan, float scale,
@@ -255,7 +245,7 @@ fca_status fca_merge_pass(fca_plan_t plan, void* out, float* lse, void* stream) 
     if (!plan || !out || !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return FCA_ERR_INVALID_ARG;
     DeviceGuard dg(plan->device);
-    return note_cuda(launch_merge(plan, out, lse, static_cast<cudaStream_t>(stream))) == cudaSuccess
+    return note_cuda(launch_merge(plan, out, lse, false, static_cast<cudaStream_t>(stream))) == cudaSuccess
                ? FCA_OK
                : FCA_ERR_CUDA;
 }

@@ -49,6 +49,16 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// The next kernel of the stream, when launched with programmatic stream
+// serialization, may start once every CTA of this grid has called this (or
+// exited).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Wait until the grids this one was launched after have completed and their
+// writes are visible (returns at once after an ordinary launch).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -157,10 +157,6 @@ struct fca_plan_s {
     int2* m_rec = nullptr;           // [R][kMergeRec] where they are: row of (KV head h, query head i)
                                      // = x + h y + i (chain order; unused when m_ng > kMergeRec)
 
-    // side stream and events for running the two passes side by side
-    cudaStream_t aux_stream = nullptr;
-    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-
     // every cudaMalloc the plan owns (freed by fca_plan_destroy)
     std::vector<void*> dev_allocs;
 };

@@ -28,6 +28,7 @@
 // few (about 8 warps per SM in all) and each has many partials to read.
 #include <cuda_bf16.h>
 
+#include "fca_device.cuh"
 #include "fca_internal.h"
 
 namespace fca {
@@ -100,6 +101,9 @@ __global__ void __launch_bounds__(256, 3) k_merge(MergeArgs a) {
     constexpr int kSlots = kSlabHeads * D / 128;   // float4 slots per lane
     constexpr int kInFlight = 2;                    // partials loaded together
     __shared__ MergeSmem<D> sm;
+    // launched after a pass with programmatic serialization: its rows are
+    // complete and visible past this point
+    dev::pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = a.W, sub = warp % W;
     const int64_t unit = (int64_t)blockIdx.x * (kWarps / W) + warp / W;
@@ -305,7 +309,10 @@ __global__ void __launch_bounds__(256, 3) k_merge(MergeArgs a) {
     }
 }
 
-cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, cudaStream_t stream) {
+// after_pass: launched right behind the pass that ends the step on the same
+// stream, with programmatic serialization, so that the grid is set up while
+// that pass runs out (its CTAs wait for it before reading a partial row).
+cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_pass, cudaStream_t stream) {
     MergeArgs a;
     a.R = P->R;
     a.Hq = P->Hq;
@@ -343,11 +350,17 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, cudaStream_
     const int64_t per_cta = kWarps / W;
     const int grid = (int)((units + per_cta - 1) / per_cta);
     if (grid == 0) return cudaSuccess;
-    if (P->D == 128)
-        k_merge<128><<<grid, 32 * kWarps, 0, stream>>>(a);
-    else
-        k_merge<64><<<grid, 32 * kWarps, 0, stream>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(32 * kWarps);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_pass ? 1 : 0;
+    return P->D == 128 ? cudaLaunchKernelEx(&cfg, k_merge<128>, a) : cudaLaunchKernelEx(&cfg, k_merge<64>, a);
 }
 
 }  // namespace fca

@@ -264,6 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 16);
     float* ml = reinterpret_cast<float*>(smem + L::kOffML);
 
+    // the per-request pass, launched after this one, may take the other SMs now
+    dev::pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t first_item = blockIdx.x, item_step = gridDim.x;
     const int32_t n_mine = first_item < a.n_items ? (a.n_items - first_item + item_step - 1) / item_step : 0;

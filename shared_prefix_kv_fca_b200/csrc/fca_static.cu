@@ -22,7 +22,7 @@ namespace fca {
 
 cudaError_t launch_suffix_devcount(const fca_plan_s* P, const void* q, const CUtensorMap& tk,
                                    const CUtensorMap& tv, float scale, cudaStream_t stream);
-cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, cudaStream_t stream);
+cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_pass, cudaStream_t stream);
 
 static_assert(FCA_STATIC_SCRATCH_BYTES == kStaticScratchBytes, "fca.h and the library disagree on the scratch size");
 
@@ -222,6 +222,6 @@ extern "C" fca_status fca_paged_decode_static(const void* q, const void* k_cache
     k_static_fill<<<(num_requests + 7) / 8, 256, 0, s>>>(f);
     if (note_cuda(cudaGetLastError()) != cudaSuccess) return FCA_ERR_CUDA;
     if (note_cuda(launch_suffix_devcount(&V, q, tk, tv, scale, s)) != cudaSuccess) return FCA_ERR_CUDA;
-    if (note_cuda(launch_merge(&V, out, lse, s)) != cudaSuccess) return FCA_ERR_CUDA;
+    if (note_cuda(launch_merge(&V, out, lse, false, s)) != cudaSuccess) return FCA_ERR_CUDA;
     return FCA_OK;
 }

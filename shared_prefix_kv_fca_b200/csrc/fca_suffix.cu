@@ -96,7 +96,12 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
         int32_t idx = 0;
         if (lane == 0) idx = atomicAdd(&a.sched[0], 1);
         idx = __shfl_sync(0xffffffffu, idx, 0);
-        if (idx >= n_items) break;
+        if (idx >= n_items) {
+            // every item is taken: the merge may be set up (it waits for this
+            // grid to end before it reads a row)
+            dev::pdl_launch_dependents();
+            break;
+        }
         const SuffixItem it = a.items[idx];
         const int32_t blk0 = it.tok0 / kBlockSize;
         const int32_t nblk = (it.tok1 + kBlockSize - 1) / kBlockSize - blk0;
@@ -289,10 +294,19 @@ __global__ void __launch_bounds__(kSufWarps * 32, 1)
             __threadfence();
         }
     }
+    // Beside the grouped pass (launched after it with programmatic
+    // serialization): end only after it, so that whatever the stream runs
+    // next sees both passes' partial rows.
+    dev::pdl_wait();
 }
 
+// beside: launched right after the grouped pass on the same stream, with
+// programmatic serialization.  The grouped pass lets it start as soon as all
+// of its CTAs run, so this grid's first CTAs take the SMs the grouped pass
+// left free and the rest take each SM the grouped pass gives up, until the
+// items run out; every CTA then waits for the grouped pass before it ends.
 template <int D, int NT, bool kDevCount = false>
-cudaError_t launch_t(const SuffixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int max_ctas,
+cudaError_t launch_t(const SuffixArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, bool beside,
                      cudaStream_t stream) {
     using L = SufLayout<D>;
     cudaError_t e =
@@ -301,10 +315,22 @@ cudaError_t launch_t(const SuffixArgs& a, const CUtensorMap& tk, const CUtensorM
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (max_ctas > 0) sms = std::min(sms, max_ctas);
     const int grid = std::max(1, std::min(sms, (a.n_items + kSufWarps - 1) / kSufWarps));
-    k_suffix<D, NT, kDevCount><<<grid, kSufWarps * 32, L::kTotal, stream>>>(a, tk, tv);
-    return cudaGetLastError();
+    if (!beside) {
+        k_suffix<D, NT, kDevCount><<<grid, kSufWarps * 32, L::kTotal, stream>>>(a, tk, tv);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kSufWarps * 32);
+    cfg.dynamicSmemBytes = L::kTotal;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_suffix<D, NT, kDevCount>, a, tk, tv);
 }
 
 SuffixArgs suffix_args(const fca_plan_s* P, const void* q, float scale) {
@@ -327,13 +353,13 @@ SuffixArgs suffix_args(const fca_plan_s* P, const void* q, float scale) {
 }  // namespace
 
 cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
-                          float scale, int max_ctas, cudaStream_t stream) {
+                          float scale, bool beside, cudaStream_t stream) {
     if (P->hdr.n_suffix_items == 0) return cudaSuccess;
     const SuffixArgs a = suffix_args(P, q, scale);
     const bool two = P->G > 8;
     if (P->D == 128)
-        return two ? launch_t<128, 2>(a, tk, tv, max_ctas, stream) : launch_t<128, 1>(a, tk, tv, max_ctas, stream);
-    return two ? launch_t<64, 2>(a, tk, tv, max_ctas, stream) : launch_t<64, 1>(a, tk, tv, max_ctas, stream);
+        return two ? launch_t<128, 2>(a, tk, tv, beside, stream) : launch_t<128, 1>(a, tk, tv, beside, stream);
+    return two ? launch_t<64, 2>(a, tk, tv, beside, stream) : launch_t<64, 1>(a, tk, tv, beside, stream);
 }
 
 cudaError_t launch_suffix_devcount(const fca_plan_s* P, const void* q, const CUtensorMap& tk,
@@ -342,8 +368,9 @@ cudaError_t launch_suffix_devcount(const fca_plan_s* P, const void* q, const CUt
     const SuffixArgs a = suffix_args(P, q, scale);
     const bool two = P->G > 8;
     if (P->D == 128)
-        return two ? launch_t<128, 2, true>(a, tk, tv, 0, stream) : launch_t<128, 1, true>(a, tk, tv, 0, stream);
-    return two ? launch_t<64, 2, true>(a, tk, tv, 0, stream) : launch_t<64, 1, true>(a, tk, tv, 0, stream);
+        return two ? launch_t<128, 2, true>(a, tk, tv, false, stream)
+                   : launch_t<128, 1, true>(a, tk, tv, false, stream);
+    return two ? launch_t<64, 2, true>(a, tk, tv, false, stream) : launch_t<64, 1, true>(a, tk, tv, false, stream);
 }
 
 }  // namespace fca
