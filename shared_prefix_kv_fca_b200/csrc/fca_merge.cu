@@ -8,24 +8,30 @@
 //     lse = log(sum_i exp(lse_i)),   out = sum_i exp(lse_i - lse) * o_i,
 // with o_i already normalised by its own softmax sum.
 //
-// Work unit: (request, KV head, slab of up to four of that KV head's query
-// heads), taken by W warps (W = 1, 2, 4 or 8, more when there are few units
-// and many partials per unit).  Every pass writes the G query heads of one
-// (request, KV head, chunk) as G consecutive partial rows, so a slab's rows of
-// one partial are one contiguous run of 4 x head_dim floats: each lane owns
-// float4 slots of that run, and the request's group chain is walked once per
-// slab, not once per query head.  The chain entries are read by one lane each
-// (all in parallel) and a warp scan turns their chunk counts into partial
-// offsets, so locating partial k costs shuffles rather than dependent loads.
-//
-// Warp w of a unit takes partials w, w + W, w + 2W, ... 32 at a time: lane i
-// locates partial i of the batch and reads its lse values; shuffle reductions
-// give each head's batch maximum and weight sum (the running state is
-// rescaled when a maximum grows); then the rows are accumulated two partials
-// at a time.  Partials with lse = -inf (empty chunks) never contribute.  With
-// W > 1 the warps' states (maximum, sum, accumulator) are combined through
-// shared memory.  A unit's warps share one CTA, so W > 1 only when units are
-// few (about 8 warps per SM in all) and each has many partials to read.
+// Every pass writes the G query heads of one (request, KV head, chunk) as G
+// consecutive partial rows.  The kernel reads a few KB per output row block,
+// each behind a lookup of where its rows lie, so it is bound by memory
+// latency and by instructions, not by bandwidth; it is laid out for two
+// rounds of loads per unit of work and few instructions per row:
+//   - a warp takes HB query heads of one (request r, KV head h): grid
+//     (R / 8, Hkv x head blocks), no division but one per warp;
+//   - lookup (first round): one lane per entry of the request's chain.  The
+//     planner records where each group partial lies (m_rec, up to kMergeRec),
+//     read together with the request's own-chunk count and first row; deeper
+//     chains (and plans without records) walk the chain, and a warp scan turns
+//     chunk counts into partial offsets;
+//   - second round: lane k loads the HB lse values of partial k and, at the
+//     same time, every lane its four columns of the first KK partials'
+//     rows; the maximum and the weight sum of each head take log2(n)
+//     shuffle steps over the n lanes that hold partials; further rows are
+//     read KK at a time.  (HB, KK) = (4, 2) for a few partials a row, (1, 8)
+//     for many.
+// Requests with more than 32 partials, or chains longer than 32 groups, take
+// a per-head loop over batches of 32 partials with a running maximum.
+// Partials with lse = -inf (empty chunks) never contribute: their rows may
+// hold anything, their weight is zero and they are not added.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 
 #include "fca_device.cuh"
@@ -34,7 +40,7 @@
 namespace fca {
 
 struct MergeArgs {
-    int32_t R, Hq, Hkv, G, n_slabs, W;
+    int32_t R, Hq, Hkv, G, n_hb;
     const int32_t* chain_off;
     const int32_t* chain_g;
     const int32_t* chain_pos;
@@ -53,21 +59,8 @@ struct MergeArgs {
 
 namespace {
 
-constexpr int kSlabHeads = 4;   // query heads per unit
-constexpr int kWarps = 8;       // warps per CTA
+constexpr int kWarps = 8;   // warps per CTA
 constexpr unsigned kFull = 0xffffffffu;
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
-    return v;
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-    return v;
-}
 
 __device__ __forceinline__ int32_t warp_incl_scan(int32_t v, int lane) {
 #pragma unroll
@@ -78,234 +71,195 @@ __device__ __forceinline__ int32_t warp_incl_scan(int32_t v, int lane) {
     return v;
 }
 
-// a[i] for a lane-dependent i, without indexing a register array at run time
-__device__ __forceinline__ float pick(const float (&a)[kSlabHeads], int i) {
-    float r = a[0];
-#pragma unroll
-    for (int k = 1; k < kSlabHeads; ++k) r = (i == k) ? a[k] : r;
-    return r;
+// Where the partial rows of (request r, KV head h) lie: entry e (held by lane
+// e) covers partials [end - nch, end), the row of head 0 of its k-th being
+// base + k * step.
+struct Entries {
+    int32_t nch, base, step, end;
+    int32_t n, depth, c0, nsc, spart;
+    bool wide;   // every entry fits one lane (else the rows are found serially)
+};
+
+__device__ __forceinline__ Entries lookup(const MergeArgs& a, int32_t r, int32_t h, int lane) {
+    Entries E;
+    E.nsc = __ldg(a.s_nch + r);
+    E.spart = __ldg(a.s_part + r);
+    const int32_t ng = a.m_ng ? __ldg(a.m_ng + r) : kMergeRec + 1;
+    // (read whatever the count is, so that it does not wait for the count)
+    const int2 rec = (a.m_rec && lane < kMergeRec) ? __ldg(a.m_rec + r * kMergeRec + lane) : make_int2(0, 0);
+    const bool recorded = ng <= kMergeRec;
+    E.c0 = recorded ? 0 : __ldg(a.chain_off + r);
+    E.depth = recorded ? ng : __ldg(a.chain_off + r + 1) - E.c0;
+    E.wide = E.depth < 32;   // warp-uniform
+    E.nch = 0;
+    E.base = 0;
+    E.step = 0;
+    if (recorded) {
+        if (lane < E.depth) {
+            E.nch = 1;
+            E.base = rec.x + h * rec.y;
+        }
+    } else if (E.wide && lane < E.depth) {
+        // group chain[e]: row of chunk k = g_part + ((h nch + k) nm + pos) G
+        const int32_t g = __ldg(a.chain_g + E.c0 + lane), pos = __ldg(a.chain_pos + E.c0 + lane);
+        const int32_t nch = __ldg(a.g_nch + g), nm = __ldg(a.g_nm + g);
+        E.nch = nch;
+        E.base = __ldg(a.g_part + g) + ((h * nch) * nm + pos) * a.G;
+        E.step = nm * a.G;
+    }
+    if (E.wide && lane == E.depth) {   // own chunks: row of chunk k = s_part + (h nsc + k) G
+        E.nch = E.nsc;
+        E.base = E.spart + h * E.nsc * a.G;
+        E.step = a.G;
+    }
+    E.end = warp_incl_scan(E.nch, lane);
+    if (E.wide) {
+        E.n = __shfl_sync(kFull, E.end, E.depth);
+    } else {   // (never for a recorded request: depth <= kMergeRec)
+        E.n = E.nsc;
+        for (int32_t c = E.c0; c < E.c0 + E.depth; ++c) E.n += __ldg(a.g_nch + __ldg(a.chain_g + c));
+    }
+    return E;
+}
+
+// Row of head 0 of partial k (any k < n; every lane calls, with its own k).
+__device__ __forceinline__ int32_t partial_row(const MergeArgs& a, const Entries& E, int32_t h, int32_t k) {
+    if (E.wide) {
+        int32_t e = 0;
+        for (int32_t x = 0; x < E.depth; ++x) e += (k >= __shfl_sync(kFull, E.end, x)) ? 1 : 0;
+        const int32_t end = __shfl_sync(kFull, E.end, e);
+        const int32_t cnt = __shfl_sync(kFull, E.nch, e);
+        const int32_t base = __shfl_sync(kFull, E.base, e);
+        const int32_t step = __shfl_sync(kFull, E.step, e);
+        return base + (k - (end - cnt)) * step;
+    }
+    if (k >= E.n) return 0;
+    for (int32_t c = E.c0; c < E.c0 + E.depth; ++c) {
+        const int32_t g = __ldg(a.chain_g + c), nch = __ldg(a.g_nch + g);
+        if (k < nch) return __ldg(a.g_part + g) + ((h * nch + k) * __ldg(a.g_nm + g) + __ldg(a.chain_pos + c)) * a.G;
+        k -= nch;
+    }
+    return E.spart + (h * E.nsc + k) * a.G;
 }
 
 template <int D>
-struct MergeSmem {
-    static constexpr int kSlots = kSlabHeads * D / 128;
-    float4 acc[kWarps][kSlots][32];
-    float m[kWarps][kSlabHeads];
-    float l[kWarps][kSlabHeads];
-};
+__device__ __forceinline__ void store_row(const MergeArgs& a, int32_t q, float4 acc, float m, float l, int lane) {
+    const float inv = l > 0.f ? __frcp_rn(l) : 0.f;
+    if (lane < D / 4) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        uint2 v;
+        v.x = *reinterpret_cast<uint32_t*>(&lo);
+        v.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(a.out + (int64_t)q * D + lane * 4) = v;
+    }
+    if (a.lse && lane == 0) a.lse[q] = l > 0.f ? m + __logf(l) : -INFINITY;
+}
+
+__device__ __forceinline__ void fma4(float4& acc, float w, const float4& v) {
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z);
+    acc.w = fmaf(w, v.w, acc.w);
+}
 
 }  // namespace
 
-template <int D>
-__global__ void __launch_bounds__(256, 3) k_merge(MergeArgs a) {
-    constexpr int kSlots = kSlabHeads * D / 128;   // float4 slots per lane
-    constexpr int kInFlight = 2;                    // partials loaded together
-    __shared__ MergeSmem<D> sm;
+template <int D, int HB, int KK>
+__global__ void __launch_bounds__(32 * kWarps, 3) k_merge(MergeArgs a) {
     // launched after a pass with programmatic serialization: its rows are
     // complete and visible past this point
     dev::pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int W = a.W, sub = warp % W;
-    const int64_t unit = (int64_t)blockIdx.x * (kWarps / W) + warp / W;
-    const bool active = unit < (int64_t)a.R * a.Hkv * a.n_slabs;   // uniform across a unit's warps
-    const int32_t slab = active ? (int32_t)(unit % a.n_slabs) : 0;
-    const int32_t rh = active ? (int32_t)(unit / a.n_slabs) : 0;
-    const int32_t r = rh / a.Hkv, h = rh % a.Hkv;
-    const int32_t gq0 = slab * kSlabHeads;
-    const int32_t nh = min(kSlabHeads, a.G - gq0);   // valid heads of this slab
+    const int32_t r = blockIdx.x * kWarps + warp;
+    if (r >= a.R) return;   // (whole warps)
+    const int32_t h = blockIdx.y / a.n_hb, gq0 = (blockIdx.y - h * a.n_hb) * HB;
+    const int32_t nh = min(HB, a.G - gq0);   // heads of this block
+    const int32_t q0 = r * a.Hq + h * a.G + gq0;   // its first output row
+    const bool cols = lane < D / 4;
+    const Entries E = lookup(a, r, h, lane);
+    const int32_t n = E.n;
 
-    // slot j of this lane: float index f = j * 128 + lane * 4 of the slab's run
-    int slot_head[kSlots];
+    if (E.wide && n <= 32) {
+        // ---- lane k < n holds partial k
+        const int32_t row = partial_row(a, E, h, lane) + gq0;
+        float lk[HB];
 #pragma unroll
-    for (int j = 0; j < kSlots; ++j) slot_head[j] = (j * 128 + lane * 4) / D;
-
-    float m[kSlabHeads], l[kSlabHeads];
+        for (int j = 0; j < HB; ++j) lk[j] = (lane < n && j < nh) ? __ldg(a.part_lse + row + j) : -INFINITY;
+        float4 o[KK][HB];
+        auto load_rows = [&](int32_t k0) {
 #pragma unroll
-    for (int i = 0; i < kSlabHeads; ++i) { m[i] = -INFINITY; l[i] = 0.f; }
-    float4 acc[kSlots];
+            for (int u = 0; u < KK; ++u) {
+                const int32_t ru = __shfl_sync(kFull, row, (k0 + u) & 31);
+                const float* src = a.part_o + (int64_t)ru * D + lane * 4;
 #pragma unroll
-    for (int j = 0; j < kSlots; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-
-    if (active) {
-        // ---- the request's partials: chain entries (one lane each), then its own chunks
-        const int32_t nsc = a.s_nch[r], spart = a.s_part[r];
-        // The planner's record of the group partials (one entry each, read
-        // with the request's own counts, no dependent loads) when it holds
-        // them all; else the chain walk.
-        const int32_t ng = a.m_ng ? a.m_ng[r] : kMergeRec + 1;
-        // (read whatever the count is, so that it does not wait for the count)
-        const int2 rec = (a.m_rec && lane < kMergeRec) ? a.m_rec[(int64_t)r * kMergeRec + lane] : make_int2(0, 0);
-        const bool recorded = ng <= kMergeRec;
-        const int32_t c0 = recorded ? 0 : a.chain_off[r];
-        const int32_t depth = recorded ? ng : a.chain_off[r + 1] - c0;
-        const bool wide = depth < 32;   // warp-uniform: every entry fits one lane
-        int32_t e_nch = 0, e_base = 0, e_step = 0;
-        if (recorded) {
-            if (lane < depth) {
-                e_nch = 1;
-                e_base = rec.x + h * rec.y + gq0;
-            } else if (lane == depth) {
-                e_nch = nsc;
-                e_base = spart + h * nsc * a.G + gq0;
-                e_step = a.G;
+                for (int j = 0; j < HB; ++j)
+                    o[u][j] = (k0 + u < n && j < nh && cols) ? __ldg(reinterpret_cast<const float4*>(src + j * D))
+                                                              : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-        } else if (wide) {
-            // entry e < depth: group chain[e]; row of (chunk k, slab) =
-            //   g_part + ((h nch + k) nm + pos) G + gq0 = e_base + k * e_step
-            // entry depth: own chunks, row = s_part + (h nsc + k) G + gq0
-            if (lane < depth) {
-                const int32_t g = a.chain_g[c0 + lane], pos = a.chain_pos[c0 + lane];
-                const int32_t nch = a.g_nch[g], nm = a.g_nm[g];
-                e_nch = nch;
-                e_base = a.g_part[g] + ((h * nch) * nm + pos) * a.G + gq0;
-                e_step = nm * a.G;
-            } else if (lane == depth) {
-                e_nch = nsc;
-                e_base = spart + h * nsc * a.G + gq0;
-                e_step = a.G;
-            }
+        };
+        load_rows(0);
+        // each head's maximum and weight sum over lanes [0, n): xor steps
+        // within the smallest power of two holding n, then from lane 0
+        float m[HB], l[HB], w[HB];
+#pragma unroll
+        for (int j = 0; j < HB; ++j) {
+            float mx = lk[j];
+            for (int s = 1; s < n; s <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, s));
+            w[j] = lk[j] == -INFINITY ? 0.f : __expf(lk[j] - mx);
+            float sm = w[j];
+            for (int s = 1; s < n; s <<= 1) sm += __shfl_xor_sync(kFull, sm, s);
+            m[j] = __shfl_sync(kFull, mx, 0);
+            l[j] = __shfl_sync(kFull, sm, 0);
         }
-        const int32_t e_end = warp_incl_scan(e_nch, lane);   // exclusive end of entry's partials
-        int32_t n = nsc;
-        if (wide) {
-            n = __shfl_sync(kFull, e_end, depth);
-        } else {   // (never for a recorded request: depth <= kMergeRec)
-            for (int32_t c = c0; c < c0 + depth; ++c) n += a.g_nch[a.chain_g[c]];
-        }
-
-        const int32_t n_mine = n > sub ? (n - sub + W - 1) / W : 0;   // partials sub, sub + W, ...
-        for (int32_t b0 = 0; b0 < n_mine; b0 += 32) {
-            // row of the slab's first head in partial k of the request (-1 past the end)
-            int32_t row = -1;
-            int32_t k = (b0 + lane) * W + sub;
-            if (wide) {
-                int32_t e = 0;
-                for (int32_t i = 0; i < depth; ++i) e += (k >= __shfl_sync(kFull, e_end, i)) ? 1 : 0;
-                const int32_t end = __shfl_sync(kFull, e_end, e);
-                const int32_t cnt = __shfl_sync(kFull, e_nch, e);
-                const int32_t base = __shfl_sync(kFull, e_base, e);
-                const int32_t step = __shfl_sync(kFull, e_step, e);
-                if (k < n) row = base + (k - (end - cnt)) * step;
-            } else if (k < n) {
-                for (int32_t c = c0; c < c0 + depth && row < 0; ++c) {
-                    const int32_t g = a.chain_g[c], nch = a.g_nch[g];
-                    if (k < nch) row = a.g_part[g] + ((h * nch + k) * a.g_nm[g] + a.chain_pos[c]) * a.G + gq0;
-                    k -= nch;
+        float4 acc[HB];
+#pragma unroll
+        for (int j = 0; j < HB; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int32_t k0 = 0; k0 < n; k0 += KK) {
+            if (k0 > 0) load_rows(k0);
+#pragma unroll
+            for (int u = 0; u < KK; ++u)
+#pragma unroll
+                for (int j = 0; j < HB; ++j) {
+                    const float wu = __shfl_sync(kFull, w[j], (k0 + u) & 31);
+                    if (k0 + u < n && wu > 0.f) fma4(acc[j], wu, o[u][j]);
                 }
-                if (row < 0) row = spart + (h * nsc + k) * a.G + gq0;
-            }
-            float li[kSlabHeads], wi[kSlabHeads], sc[kSlabHeads];
-#pragma unroll
-            for (int i = 0; i < kSlabHeads; ++i)
-                li[i] = (row >= 0 && i < nh) ? __ldg(a.part_lse + row + i) : -INFINITY;
-#pragma unroll
-            for (int i = 0; i < kSlabHeads; ++i) {
-                const float m_new = fmaxf(m[i], warp_max(li[i]));
-                sc[i] = m_new == -INFINITY ? 1.f : expf(m[i] - m_new);   // 0 while nothing has been added
-                wi[i] = li[i] == -INFINITY ? 0.f : expf(li[i] - m_new);
-                l[i] = l[i] * sc[i] + warp_sum(wi[i]);
-                m[i] = m_new;
-            }
-#pragma unroll
-            for (int j = 0; j < kSlots; ++j) {
-                const float s = pick(sc, slot_head[j]);
-                acc[j].x *= s; acc[j].y *= s; acc[j].z *= s; acc[j].w *= s;
-            }
-            const int32_t nb = min(32, n_mine - b0);
-            for (int32_t j0 = 0; j0 < nb; j0 += kInFlight) {
-                float4 o[kInFlight][kSlots];
-                float w[kInFlight][kSlots];
-#pragma unroll
-                for (int u = 0; u < kInFlight; ++u) {
-                    const int32_t jj = (j0 + u) & 31;
-                    const int32_t rj = __shfl_sync(kFull, row, jj);
-                    float wh[kSlabHeads];
-#pragma unroll
-                    for (int i = 0; i < kSlabHeads; ++i) wh[i] = __shfl_sync(kFull, wi[i], jj);
-                    const float* src = a.part_o + (int64_t)rj * D + lane * 4;
-#pragma unroll
-                    for (int j = 0; j < kSlots; ++j) {
-                        w[u][j] = (j0 + u < nb && slot_head[j] < nh) ? pick(wh, slot_head[j]) : 0.f;
-                        o[u][j] = w[u][j] > 0.f ? __ldg(reinterpret_cast<const float4*>(src + j * 128))
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < kInFlight; ++u)
-#pragma unroll
-                    for (int j = 0; j < kSlots; ++j) {
-                        acc[j].x = fmaf(w[u][j], o[u][j].x, acc[j].x);
-                        acc[j].y = fmaf(w[u][j], o[u][j].y, acc[j].y);
-                        acc[j].z = fmaf(w[u][j], o[u][j].z, acc[j].z);
-                        acc[j].w = fmaf(w[u][j], o[u][j].w, acc[j].w);
-                    }
-            }
         }
+#pragma unroll
+        for (int j = 0; j < HB; ++j)
+            if (j < nh) store_row<D>(a, q0 + j, acc[j], m[j], l[j], lane);
+        return;
     }
 
-    // ---- combine the W warps of a unit (W is uniform across the CTA)
-    if (W > 1) {
+    // ---- many partials or a deep chain: one head at a time, batches of 32
+    for (int j = 0; j < nh; ++j) {
+        float m = -INFINITY, l = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int32_t b0 = 0; b0 < n; b0 += 32) {
+            const int32_t k = b0 + lane;
+            const int32_t row = partial_row(a, E, h, k) + gq0 + j;
+            const float lk = k < n ? __ldg(a.part_lse + row) : -INFINITY;
+            float mb = lk;
 #pragma unroll
-        for (int j = 0; j < kSlots; ++j) sm.acc[warp][j][lane] = acc[j];
-        if (lane < kSlabHeads) {
-            sm.m[warp][lane] = pick(m, lane);
-            sm.l[warp][lane] = pick(l, lane);
-        }
-        __syncthreads();
-        if (sub != 0) return;
+            for (int s = 16; s > 0; s >>= 1) mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, s));
+            const float m_new = fmaxf(m, mb);
+            const float sc = m_new == -INFINITY ? 1.f : __expf(m - m_new);   // 0 while nothing has been added
+            const float w = lk == -INFINITY ? 0.f : __expf(lk - m_new);
+            float ws = w;
 #pragma unroll
-        for (int i = 0; i < kSlabHeads; ++i) {
-            float mm = -INFINITY;
-            for (int v = 0; v < W; ++v) mm = fmaxf(mm, sm.m[warp + v][i]);
-            float ll = 0.f;
-            for (int v = 0; v < W; ++v) {
-                const float mv = sm.m[warp + v][i];
-                ll += mv == -INFINITY ? 0.f : sm.l[warp + v][i] * expf(mv - mm);
-            }
-            m[i] = mm;
-            l[i] = ll;
-        }
-#pragma unroll
-        for (int j = 0; j < kSlots; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int v = 0; v < W; ++v) {
-            float f[kSlabHeads];
-#pragma unroll
-            for (int i = 0; i < kSlabHeads; ++i) {
-                const float mv = sm.m[warp + v][i];
-                f[i] = mv == -INFINITY ? 0.f : expf(mv - m[i]);
-            }
-#pragma unroll
-            for (int j = 0; j < kSlots; ++j) {
-                const float s = pick(f, slot_head[j]);
-                const float4 x = sm.acc[warp + v][j][lane];
-                acc[j].x = fmaf(s, x.x, acc[j].x);
-                acc[j].y = fmaf(s, x.y, acc[j].y);
-                acc[j].z = fmaf(s, x.z, acc[j].z);
-                acc[j].w = fmaf(s, x.w, acc[j].w);
+            for (int s = 16; s > 0; s >>= 1) ws += __shfl_xor_sync(kFull, ws, s);
+            l = l * sc + ws;
+            m = m_new;
+            acc.x *= sc; acc.y *= sc; acc.z *= sc; acc.w *= sc;
+            const int32_t nb = min(32, n - b0);
+            for (int32_t u = 0; u < nb; ++u) {
+                const int32_t ru = __shfl_sync(kFull, row, u);
+                const float wu = __shfl_sync(kFull, w, u);
+                if (wu > 0.f && cols)
+                    fma4(acc, wu, __ldg(reinterpret_cast<const float4*>(a.part_o + (int64_t)ru * D + lane * 4)));
             }
         }
-    }
-    if (!active) return;
-
-    // ---- normalise and store: out[r][h G + gq0 + head][col], lse[r][h G + gq0 + head]
-    float inv[kSlabHeads];
-#pragma unroll
-    for (int i = 0; i < kSlabHeads; ++i) inv[i] = l[i] > 0.f ? 1.f / l[i] : 0.f;
-    const int64_t q0 = (int64_t)r * a.Hq + (int64_t)h * a.G + gq0;   // first query head of the slab
-#pragma unroll
-    for (int j = 0; j < kSlots; ++j) {
-        if (slot_head[j] >= nh) continue;
-        const float s = pick(inv, slot_head[j]);
-        uint2 v;
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j].x * s, acc[j].y * s);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j].z * s, acc[j].w * s);
-        v.x = *reinterpret_cast<uint32_t*>(&lo);
-        v.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(a.out + q0 * D + j * 128 + lane * 4) = v;
-    }
-    if (a.lse && lane < nh) {
-        const float mm = pick(m, lane), ll = pick(l, lane);
-        a.lse[q0 + lane] = ll > 0.f ? mm + logf(ll) : -INFINITY;
+        store_row<D>(a, q0 + j, acc, m, l, lane);
     }
 }
 
@@ -318,7 +272,6 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_
     a.Hq = P->Hq;
     a.Hkv = P->Hkv;
     a.G = P->G;
-    a.n_slabs = (P->G + kSlabHeads - 1) / kSlabHeads;
     a.chain_off = P->chain_off;
     a.chain_g = P->chain_g;
     a.chain_pos = P->chain_pos;
@@ -333,25 +286,15 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_
     a.lse = lse;
     a.m_ng = P->m_ng;
     a.m_rec = P->m_rec;
-    const int64_t units = (int64_t)P->R * P->Hkv * a.n_slabs;
-    // Warps per unit: split a unit's partials over more warps only while the
-    // whole grid stays under about 8 warps per SM and every warp still gets
-    // two partials or more on average (a sweep of 8, 16 and 32 warps per SM on
-    // the four large workloads favoured 8: extra warps per unit cost more in
-    // the combine than they save when units are plentiful).
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (P->R == 0) return cudaSuccess;
+    // partials per output row on average: many -> one head a warp, eight rows in flight
     const int64_t pairs = (int64_t)P->R * P->Hq;
     const int64_t n_part = (int64_t)P->hdr.n_prefix_partials + P->hdr.n_suffix_partials;
-    const double per_pair = pairs > 0 ? (double)n_part / (double)pairs : 0.0;
-    int W = 1;
-    while (W < kWarps && units * W < (int64_t)sms * 8 && 2.0 * W <= per_pair) W *= 2;
-    a.W = W;
-    const int64_t per_cta = kWarps / W;
-    const int grid = (int)((units + per_cta - 1) / per_cta);
-    if (grid == 0) return cudaSuccess;
+    const bool many = pairs > 0 && n_part > 4 * pairs;
+    const int hb = many ? 1 : 4;
+    a.n_hb = (P->G + hb - 1) / hb;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
+    cfg.gridDim = dim3((unsigned)((P->R + kWarps - 1) / kWarps), (unsigned)(P->Hkv * a.n_hb));
     cfg.blockDim = dim3(32 * kWarps);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
@@ -360,7 +303,9 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = after_pass ? 1 : 0;
-    return P->D == 128 ? cudaLaunchKernelEx(&cfg, k_merge<128>, a) : cudaLaunchKernelEx(&cfg, k_merge<64>, a);
+    if (P->D == 128)
+        return many ? cudaLaunchKernelEx(&cfg, k_merge<128, 1, 8>, a) : cudaLaunchKernelEx(&cfg, k_merge<128, 4, 2>, a);
+    return many ? cudaLaunchKernelEx(&cfg, k_merge<64, 1, 8>, a) : cudaLaunchKernelEx(&cfg, k_merge<64, 4, 2>, a);
 }
 
 }  // namespace fca
