@@ -88,6 +88,13 @@ typedef struct fca_plan_opts {
  * pass.  fca_decode on such a plan is the flat (non-cascaded) paged decode. */
 #define FCA_PLAN_FLAT 1u
 
+/* Let fca_plan_update run without synchronising the host: the plan reserves,
+ * when it is built, own-pass room for the longest request the tables can hold
+ * (each request's table width past its shared blocks, in chunks of at least
+ * 512 tokens, or split_tokens when set), and each update is checked, sized
+ * and applied on the device.  See fca_plan_update for what changes. */
+#define FCA_PLAN_ASYNC_UPDATE 2u
+
 /* Default options (min_group_size 2, min_shared_blocks 1, split auto, flags 0,
  * min_saved_blocks 32). */
 void fca_plan_opts_default(fca_plan_opts *opts /* HOST, out */);
@@ -142,7 +149,15 @@ fca_status fca_plan(const int32_t *block_tables, int32_t max_blocks, const int32
  * of the previous step has been queued there.
  *
  * Synchronises `stream` once (the new sizes), like fca_plan; may take more
- * memory from the plan pool if the own work outgrew the plan.  Errors:
+ * memory from the plan pool if the own work outgrew the plan.
+ *
+ * A plan built with FCA_PLAN_ASYNC_UPDATE is updated without any host
+ * synchronisation: the checks below run on the device, a refused update
+ * leaves the plan as it was and records kErrUpdateRefused (32) in the plan's
+ * device status (fca_check_device_status), and the function returns FCA_OK
+ * as soon as the work is queued; block_tables and seq_lens must stay valid
+ * until `stream` has run it.  fca_plan_get_stats then keeps describing the
+ * plan as built.  Errors (synchronous plans):
  * FCA_ERR_INVALID_ARG (a shared entry changed, a length no longer covers the
  * shared blocks or is out of range, another table shape), FCA_ERR_BAD_BLOCK_ID,
  * FCA_ERR_UNSUPPORTED (more partial rows than the planner indexes),

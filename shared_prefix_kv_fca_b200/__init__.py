@@ -28,7 +28,7 @@ __all__ = [
     "fca_plan_export", "fca_plan_member_count", "fca_plan_destroy", "fca_check_device_status",
     "fca_status_string", "fca_version", "fca_plan_opts_default", "library_path", "load_library",
     "fca_prefix_pass", "fca_suffix_pass", "fca_merge_pass", "fca_last_cuda_error",
-    "FCA_PLAN_FLAT", "STATUS", "fca_paged_decode_static", "FCA_STATIC_SCRATCH_BYTES",
+    "FCA_PLAN_FLAT", "FCA_PLAN_ASYNC_UPDATE", "STATUS", "fca_paged_decode_static", "FCA_STATIC_SCRATCH_BYTES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +36,7 @@ _LIB_PATH = os.path.join(_HERE, "libfca_b200.so")
 _lib = None
 
 FCA_PLAN_FLAT = 1
+FCA_PLAN_ASYNC_UPDATE = 2
 STATUS = {0: "FCA_OK", 1: "FCA_ERR_INVALID_ARG", 2: "FCA_ERR_BAD_BLOCK_ID", 3: "FCA_ERR_UNSUPPORTED",
           4: "FCA_ERR_CUDA", 5: "FCA_ERR_OOM", 6: "FCA_ERR_DEVICE_FLAG", 7: "FCA_ERR_TOO_LARGE"}
 FCA_STATIC_SCRATCH_BYTES = 64 << 20
@@ -228,16 +229,19 @@ def fca_plan_opts_default() -> fca_plan_opts:
 def fca_plan(block_tables, seq_lens, num_blocks: int, num_q_heads: int, num_kv_heads: int,
              head_dim: int, block_size: int = 16, min_group_size: int = 2,
              min_shared_blocks: int = 1, split_tokens: int = 0, flat: bool = False,
-             stream=None, min_saved_blocks: int = 32) -> "Plan":
+             stream=None, min_saved_blocks: int = 32, async_update: bool = False) -> "Plan":
     """Group discovery + work lists.  block_tables int32 [R, max_blocks] and
     seq_lens int32 [R] are CUDA tensors.  min_saved_blocks: groups whose
     sharing saves fewer block reads ((members - 1) x length in blocks) are
-    folded (0 keeps every shared prefix)."""
+    folded (0 keeps every shared prefix).  async_update: FCA_PLAN_ASYNC_UPDATE
+    (Plan.update queues its work without synchronising the host; a refused
+    update shows in fca_check_device_status)."""
     lib = load_library()
     _check_tables(block_tables, seq_lens)
     dev = _one_device(("block_tables", block_tables), ("seq_lens", seq_lens))
     R, mb = block_tables.shape
-    o = fca_plan_opts(min_group_size, min_shared_blocks, split_tokens, FCA_PLAN_FLAT if flat else 0,
+    o = fca_plan_opts(min_group_size, min_shared_blocks, split_tokens,
+                      (FCA_PLAN_FLAT if flat else 0) | (FCA_PLAN_ASYNC_UPDATE if async_update else 0),
                       min_saved_blocks)
     handle = ctypes.c_void_p()
     with _on_device(dev):       # the plan belongs to the device current when it is built

@@ -137,6 +137,7 @@ fca_status fca_plan(const int32_t* block_tables, int32_t max_blocks, const int32
     P->G = num_q_heads / num_kv_heads;
     P->opts = o;
     P->flat = (o.flags & FCA_PLAN_FLAT) != 0;
+    P->async_update = (o.flags & FCA_PLAN_ASYNC_UPDATE) != 0;
     const fca_status st = plan_build(block_tables, seq_lens, static_cast<cudaStream_t>(stream), P);
     if (st != FCA_OK) {
         fca_plan_destroy(P);
@@ -189,7 +190,7 @@ static fca_status decode_impl(const void* q, const void* k_cache, const void* v_
         !make_cache_map(&tv, v_cache, plan->num_blocks, plan->Hkv, plan->D))
         return FCA_ERR_CUDA;
     const bool grouped = !plan->flat && plan->hdr.n_prefix_items > 0;
-    const bool own = plan->hdr.n_suffix_items > 0;
+    const bool own = plan->async_update ? plan->cap_suffix_items > 0 : plan->hdr.n_suffix_items > 0;
     if (grouped) {
         // The two passes are independent.  With both, they share the SMs: the
         // grouped pass on its share, the per-request pass on the rest and then

@@ -24,6 +24,7 @@ constexpr int kMaxRequestsFallback = 4096;  // all-pairs LCP path (see fca_plan.
 constexpr int32_t kErrWaitTimeout = 1;     // a bounded mbarrier wait ran out
 constexpr int32_t kErrBadItem = 2;         // a work item failed its own range check
 constexpr int32_t kErrPlanInternal = 4;    // a planner consistency check failed (no write done)
+constexpr int32_t kErrUpdateRefused = 32;  // an asynchronous fca_plan_update was refused (plan unchanged)
 
 // Raised by the work-list kernel of fca_paged_decode_static, which cannot
 // return an error to the host: the request is skipped (out 0, lse -inf).
@@ -101,6 +102,7 @@ struct PlanHeader {
     int64_t prefix_tok_sum;     // sum over groups of their token count
     int64_t suffix_tok_sum;
     int64_t prefix_tile_tok_sum;// sum over groups of token count x 128-row query tiles
+    int64_t own_chunk_cap;      // own-pass chunks any update can need (plans with asynchronous updates)
 };
 
 // Remember e (if it is an error) as the calling thread's last CUDA error.
@@ -124,6 +126,8 @@ struct fca_plan_s {
     size_t workspace_bytes = 0;
     int64_t cap_suffix_items = 0;    // capacity of suffix_items (fca_plan_update may need more)
     int64_t cap_partials = 0;        // capacity of part_o / part_lse, in rows
+    bool async_update = false;       // FCA_PLAN_ASYNC_UPDATE: updates stay on the device; the
+                                     // per-request pass reads its item count from sched[2]
 
     // copies of the inputs
     int32_t* bt = nullptr;           // [R][max_blocks]

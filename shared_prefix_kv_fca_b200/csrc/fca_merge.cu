@@ -59,7 +59,8 @@ struct MergeArgs {
 
 namespace {
 
-constexpr int kWarps = 8;   // warps per CTA
+constexpr int kWarps = 8;       // warps per CTA
+constexpr int kCtasPerSM = 3;   // resident CTAs per SM (the persistent grid)
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ int32_t warp_incl_scan(int32_t v, int lane) {
@@ -165,15 +166,9 @@ __device__ __forceinline__ void fma4(float4& acc, float w, const float4& v) {
 
 }  // namespace
 
+// Query heads gq0 .. gq0 + HB - 1 of (request r, KV head h): one warp.
 template <int D, int HB, int KK>
-__global__ void __launch_bounds__(32 * kWarps, 3) k_merge(MergeArgs a) {
-    // launched after a pass with programmatic serialization: its rows are
-    // complete and visible past this point
-    dev::pdl_wait();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int32_t r = blockIdx.x * kWarps + warp;
-    if (r >= a.R) return;   // (whole warps)
-    const int32_t h = blockIdx.y / a.n_hb, gq0 = (blockIdx.y - h * a.n_hb) * HB;
+__device__ __forceinline__ void merge_unit(const MergeArgs& a, int32_t r, int32_t h, int32_t gq0, int lane) {
     const int32_t nh = min(HB, a.G - gq0);   // heads of this block
     const int32_t q0 = r * a.Hq + h * a.G + gq0;   // its first output row
     const bool cols = lane < D / 4;
@@ -263,6 +258,23 @@ __global__ void __launch_bounds__(32 * kWarps, 3) k_merge(MergeArgs a) {
     }
 }
 
+template <int D, int HB, int KK>
+__global__ void __launch_bounds__(32 * kWarps, kCtasPerSM) k_merge(MergeArgs a) {
+    // launched after a pass with programmatic serialization: its rows are
+    // complete and visible past this point
+    dev::pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // persistent: warp w takes units w, w + all warps, ...; unit u is head
+    // block y = u mod Y of request u / Y, Y = Hkv x head blocks (a request's
+    // units on neighbouring warps)
+    const int32_t Y = a.Hkv * a.n_hb, n_units = a.R * Y;
+    for (int32_t u = blockIdx.x * kWarps + warp; u < n_units; u += gridDim.x * kWarps) {
+        const int32_t r = u / Y, y = u - r * Y;
+        const int32_t h = y / a.n_hb;
+        merge_unit<D, HB, KK>(a, r, h, (y - h * a.n_hb) * HB, lane);
+    }
+}
+
 // after_pass: launched right behind the pass that ends the step on the same
 // stream, with programmatic serialization, so that the grid is set up while
 // that pass runs out (its CTAs wait for it before reading a partial row).
@@ -294,7 +306,10 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_
     const int hb = many ? 1 : 4;
     a.n_hb = (P->G + hb - 1) / hb;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((P->R + kWarps - 1) / kWarps), (unsigned)(P->Hkv * a.n_hb));
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t units = (int64_t)P->R * P->Hkv * a.n_hb;
+    cfg.gridDim = dim3((unsigned)std::min<int64_t>((units + kWarps - 1) / kWarps, (int64_t)sms * kCtasPerSM));
     cfg.blockDim = dim3(32 * kWarps);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;

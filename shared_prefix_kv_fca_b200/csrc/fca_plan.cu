@@ -754,9 +754,36 @@ __global__ void k_fill_prefix_items(const PlanHeader* hdr, const int32_t* g_wa, 
     }
 }
 
+// Own-pass chunks that any update of a plan can need: request r's own range
+// can grow to the table's width past its shared blocks, in chunks of at least
+// min_chunk tokens (the update's chunk target never goes below it).
+__global__ void __launch_bounds__(1024) k_own_cap(int32_t R, int32_t max_blocks, const int32_t* suffix_start,
+                                                  int32_t min_chunk, PlanHeader* hdr) {
+    __shared__ int64_t red[64];
+    int64_t c = 0;
+    for (int32_t r = threadIdx.x; r < R; r += blockDim.x) {
+        const int64_t tok = (int64_t)(max_blocks - suffix_start[r]) * kBlockSize;
+        c += (tok + min_chunk - 1) / min_chunk;
+    }
+    c = block_sum64(c, red);
+    if (threadIdx.x == 0) hdr->own_chunk_cap = c;
+}
+
+// An asynchronous update goes ahead only if every check passed and its own
+// work fits the room the plan reserved.
+__device__ __forceinline__ bool update_fits(const PlanHeader* hdr, int64_t cap_items, int64_t cap_rows,
+                                            int64_t n_ppart) {
+    return hdr->status == 0 && hdr->n_suffix_items <= cap_items && n_ppart + hdr->n_suffix_partials <= cap_rows;
+}
+
+// gate: null, or the header of an asynchronous update, which writes the
+// items only if it fits (update_fits).
 __global__ void k_fill_suffix_items(int32_t R, const int32_t* seq_lens, const int32_t* suffix_start,
                                     const int32_t* s_nch, const int32_t* s_chunk, const int32_t* s_part,
-                                    int32_t* bin_cursor, int32_t G, int32_t Hkv, SuffixItem* items) {
+                                    int32_t* bin_cursor, int32_t G, int32_t Hkv, SuffixItem* items,
+                                    const PlanHeader* gate = nullptr, int64_t cap_items = 0,
+                                    int64_t cap_rows = 0, int64_t n_ppart = 0) {
+    if (gate && !update_fits(gate, cap_items, cap_rows, n_ppart)) return;
     // one thread per request; the Hkv heads of one chunk take consecutive
     // slots (one DRAM row holds all heads of a token, so they should run together)
     for (int32_t r = blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x) {
@@ -1131,6 +1158,12 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     k_finalize<<<1, 1024, fin_smem, stream>>>(fa);
     FCA_CK(cudaGetLastError());
 
+    if (P->async_update) {
+        const int32_t min_chunk = opts.split_tokens > 0 ? opts.split_tokens : kMinOwnChunk;
+        k_own_cap<<<1, 1024, 0, stream>>>(R, max_blocks, P->suffix_start, min_chunk, s.hdr);
+        FCA_CK(cudaGetLastError());
+    }
+
     // the one synchronisation: sizes of the forest and of the work lists
     FCA_CK(cudaMemcpyAsync(&P->hdr, s.hdr, sizeof(PlanHeader), cudaMemcpyDeviceToHost, stream));
     FCA_CK(cudaStreamSynchronize(stream));
@@ -1139,7 +1172,10 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     if (H.status & kPlanBadBlockId) return FCA_ERR_BAD_BLOCK_ID;
     if (H.status & kPlanTooManyGroups) return FCA_ERR_UNSUPPORTED;
     if ((H.status & kPlanInconsistent) && R > kMaxRequestsFallback) return FCA_ERR_UNSUPPORTED;
-    const int64_t n_part = (int64_t)H.n_prefix_partials + H.n_suffix_partials;
+    // own-pass room: what this plan needs, or (asynchronous updates) what any update can
+    const int64_t cap_items =
+        P->async_update ? std::max<int64_t>(H.n_suffix_items, (int64_t)Hkv * H.own_chunk_cap) : H.n_suffix_items;
+    const int64_t n_part = (int64_t)H.n_prefix_partials + cap_items * G;
     if (n_part >= (int64_t)INT32_MAX / 2) return FCA_ERR_UNSUPPORTED;
 
     // the arrays sized by the planner
@@ -1148,7 +1184,7 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     wa.add(&P->chain_g, H.n_chain_entries);
     wa.add(&P->chain_pos, H.n_chain_entries);
     wa.add(&P->prefix_items, H.n_prefix_items);
-    wa.add(&P->suffix_items, H.n_suffix_items);
+    wa.add(&P->suffix_items, cap_items);
     wa.add(&P->part_lse, n_part);
     wa.add(&P->part_o, (size_t)n_part * D);
     {
@@ -1159,9 +1195,12 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
         }
         P->dev_allocs.push_back(base);
         P->workspace_bytes += wa.bytes;
-        P->cap_suffix_items = H.n_suffix_items;
+        P->cap_suffix_items = cap_items;
         P->cap_partials = n_part;
     }
+    if (P->async_update)   // the per-request pass's item count, read on the device
+        FCA_CK(cudaMemcpyAsync(P->sched + 2, &P->hdr.n_suffix_items, sizeof(int32_t), cudaMemcpyHostToDevice,
+                               stream));
 
     if (!flat && H.n_groups > 0) {
         ra.pass = 1;
@@ -1190,6 +1229,44 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
                                                           P->g_nm, P->g_part, P->m_ng, P->m_rec);
     FCA_CK(cudaGetLastError());
     return FCA_OK;   // temporaries go back to the pool in stream order
+}
+
+// Applies an asynchronous update on the device: the new tables, lengths and
+// own-pass arrays replace the plan's, and the per-request pass's item count
+// (sched[2]) is set, if the update fits; otherwise nothing changes and the
+// plan's status word records kErrUpdateRefused.
+struct UpdateApplyArgs {
+    const PlanHeader* hdr;
+    int64_t cap_items, cap_rows, n_ppart, cells;
+    int32_t R;
+    const int32_t* bt_new;
+    const int32_t* sl_new;
+    const int32_t* t_nch;
+    const int32_t* t_chunk;
+    const int32_t* t_part;
+    int32_t* bt;
+    int32_t* seq_lens;
+    int32_t* s_nch;
+    int32_t* s_chunk;
+    int32_t* s_part;
+    int32_t* sched;
+    int32_t* err;
+};
+
+__global__ void k_update_apply(UpdateApplyArgs A) {
+    if (!update_fits(A.hdr, A.cap_items, A.cap_rows, A.n_ppart)) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(A.err, kErrUpdateRefused);
+        return;
+    }
+    const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x, step = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = t0; i < A.cells; i += step) A.bt[i] = A.bt_new[i];
+    for (int64_t r = t0; r < A.R; r += step) {
+        A.seq_lens[r] = A.sl_new[r];
+        A.s_nch[r] = A.t_nch[r];
+        A.s_chunk[r] = A.t_chunk[r];
+    }
+    for (int64_t r = t0; r <= A.R; r += step) A.s_part[r] = A.t_part[r];
+    if (t0 == 0) A.sched[2] = A.hdr->n_suffix_items;
 }
 
 // Next decode step of the same batch: new lengths (and tables grown past the
@@ -1255,6 +1332,36 @@ fca_status plan_update(const int32_t* block_tables, const int32_t* seq_lens, cud
     const size_t upd_smem = (64 + 1024) * 8 + kBins * 4;
     k_update_own<<<1, 1024, upd_smem, stream>>>(ua);
     FCA_CK(cudaGetLastError());
+
+    if (P->async_update) {
+        // checked, sized and applied on the device; no host synchronisation
+        UpdateApplyArgs ap{};
+        ap.hdr = hdr;
+        ap.cap_items = P->cap_suffix_items;
+        ap.cap_rows = P->cap_partials;
+        ap.n_ppart = P->hdr.n_prefix_partials;
+        ap.cells = cells;
+        ap.R = R;
+        ap.bt_new = block_tables;
+        ap.sl_new = seq_lens;
+        ap.t_nch = t_nch;
+        ap.t_chunk = t_chunk;
+        ap.t_part = t_part;
+        ap.bt = P->bt;
+        ap.seq_lens = P->seq_lens;
+        ap.s_nch = P->s_nch;
+        ap.s_chunk = P->s_chunk;
+        ap.s_part = P->s_part;
+        ap.sched = P->sched;
+        ap.err = P->dev_status;
+        k_update_apply<<<grid_for(cells, 256), 256, 0, stream>>>(ap);
+        k_fill_suffix_items<<<grid_for(R, 128), 128, 0, stream>>>(R, P->seq_lens, P->suffix_start, P->s_nch,
+                                                                  P->s_chunk, P->s_part, bin_cursor, G, Hkv,
+                                                                  P->suffix_items, hdr, P->cap_suffix_items,
+                                                                  P->cap_partials, P->hdr.n_prefix_partials);
+        FCA_CK(cudaGetLastError());
+        return FCA_OK;   // temporaries go back to the pool in stream order
+    }
 
     PlanHeader H{};
     FCA_CK(cudaMemcpyAsync(&H, hdr, sizeof(PlanHeader), cudaMemcpyDeviceToHost, stream));

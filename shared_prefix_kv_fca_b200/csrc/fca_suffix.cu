@@ -354,6 +354,18 @@ SuffixArgs suffix_args(const fca_plan_s* P, const void* q, float scale) {
 
 cudaError_t launch_suffix(const fca_plan_s* P, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
                           float scale, bool beside, cudaStream_t stream) {
+    if (P->async_update) {
+        // the item count of the last update is on the device (sched[2]);
+        // the grid is sized for the plan's room
+        if (P->cap_suffix_items == 0) return cudaSuccess;
+        SuffixArgs a = suffix_args(P, q, scale);
+        a.n_items = (int32_t)std::min<int64_t>(P->cap_suffix_items, INT32_MAX);
+        const bool two = P->G > 8;
+        if (P->D == 128)
+            return two ? launch_t<128, 2, true>(a, tk, tv, beside, stream)
+                       : launch_t<128, 1, true>(a, tk, tv, beside, stream);
+        return two ? launch_t<64, 2, true>(a, tk, tv, beside, stream) : launch_t<64, 1, true>(a, tk, tv, beside, stream);
+    }
     if (P->hdr.n_suffix_items == 0) return cudaSuccess;
     const SuffixArgs a = suffix_args(P, q, scale);
     const bool two = P->G > 8;

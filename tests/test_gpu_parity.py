@@ -665,3 +665,99 @@ def test_plan_update_full_size_one_token_steps():
         assert_plan_equal(ref, oracle.plan(cur.block_tables, cur.seq_lens, 16, min_saved_blocks=32))
         o, l = decode_with(plan, cur)
     assert_all_vs_oracle(cur, o, l, "llama8b after 20 updates")
+
+
+# ---- plans with asynchronous updates (FCA_PLAN_ASYNC_UPDATE): the same
+# growth, checked and applied on the device without a host synchronisation
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("split", [0, 64])
+def test_plan_update_async_follows_growing_requests(seed, split):
+    import shared_prefix_kv_fca_b200 as fca
+    w0 = fca_workloads.random_small(seed, max_requests=24)
+    base, steps = growth_steps(w0, seed)
+    bt, sl = base.torch_inputs("cuda")[3:]
+    ref = oracle.plan(base.block_tables, base.seq_lens, 16)
+    with fca.fca_plan(bt, sl, base.num_blocks, w0.Hq, w0.Hkv, w0.D, min_saved_blocks=0,
+                      split_tokens=split, async_update=True) as plan:
+        assert_plan_equal(plan.export(), ref)
+        check_all(plan, base, f"async seed {seed} step 0")
+        for s, cur in enumerate(steps):
+            bt2, sl2 = cur.torch_inputs("cuda")[3:]
+            plan.update(bt2, sl2)
+            check_all(plan, cur, f"async seed {seed} step {s + 1}")
+            assert_plan_equal(plan.export(), ref)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_plan_update_async_flat(seed):
+    import shared_prefix_kv_fca_b200 as fca
+    w0 = fca_workloads.random_small(seed, max_requests=24)
+    base, steps = growth_steps(w0, seed, n_steps=2)
+    bt, sl = base.torch_inputs("cuda")[3:]
+    with fca.fca_plan(bt, sl, base.num_blocks, w0.Hq, w0.Hkv, w0.D, flat=True, async_update=True) as plan:
+        check_all(plan, base, f"async flat seed {seed} step 0", flat=True)
+        for s, cur in enumerate(steps):
+            bt2, sl2 = cur.torch_inputs("cuda")[3:]
+            plan.update(bt2, sl2)
+            check_all(plan, cur, f"async flat seed {seed} step {s + 1}", flat=True)
+
+
+def test_plan_update_async_refusal_is_recorded_and_leaves_the_plan():
+    # a refused asynchronous update returns at once; the plan's device status
+    # records it (bit 32) and the plan still decodes the batch it last had
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    for seed in range(40):
+        w0 = fca_workloads.random_small(seed, max_requests=24)
+        ref = oracle.plan(w0.block_tables, w0.seq_lens, 16)
+        if w0.R >= 2 and ref["suffix_start"].max() > 1:
+            break
+    base, (nxt,) = growth_steps(w0, seed, n_steps=1)
+    r = int(np.argmax(ref["suffix_start"]))
+    ss = int(ref["suffix_start"][r])
+    bt, sl = base.torch_inputs("cuda")[3:]
+    with fca.fca_plan(bt, sl, base.num_blocks, w0.Hq, w0.Hkv, w0.D, min_saved_blocks=0,
+                      async_update=True) as plan:
+        replaced = nxt.block_tables.copy()
+        replaced[r, ss - 1] = base.num_blocks - 1    # a shared entry replaced
+        short = nxt.seq_lens.copy()
+        short[r] = ss * 16 - 1                       # the request no longer covers its groups
+        for bad_bt, bad_sl in ((replaced, nxt.seq_lens), (nxt.block_tables, short)):
+            bt_t = torch.from_numpy(np.ascontiguousarray(bad_bt, np.int32)).cuda()
+            sl_t = torch.from_numpy(np.ascontiguousarray(bad_sl, np.int32)).cuda()
+            plan.update(bt_t, sl_t)              # queued, no status yet
+            with pytest.raises(fca.FcaError) as ei:
+                fca.fca_check_device_status(plan)
+            assert "0x20" in str(ei.value)
+            check_all(plan, base, "after a refused asynchronous update")
+        bt2, sl2 = nxt.torch_inputs("cuda")[3:]
+        plan.update(bt2, sl2)
+        check_all(plan, nxt, "after the good asynchronous update")
+
+
+def test_plan_update_async_full_size_one_token_steps():
+    # the llama8b decode loop with an asynchronous plan: 20 one-token steps
+    # queued back to back, one check at the end
+    import shared_prefix_kv_fca_b200 as fca
+    w0 = fca_workloads.make("llama8b")
+    B = 16
+    n_steps = 20
+    final = w0.seq_lens.astype(np.int64) + n_steps
+    need = int(((final + B - 1) // B - (w0.seq_lens.astype(np.int64) + B - 1) // B).sum())
+    base = pooled(w0, need, int(((final + B - 1) // B).max()), 0)
+    q, k, v, bt, sl = base.torch_inputs("cuda")
+    cur = base
+    keep = []
+    with fca.fca_plan(bt, sl, base.num_blocks, w0.Hq, w0.Hkv, w0.D, async_update=True) as plan:
+        taken = 0
+        for s in range(n_steps):
+            nb_before = (cur.seq_lens.astype(np.int64) + B - 1) // B
+            cur = grown(cur, np.ones(w0.R, np.int64), w0.num_blocks + taken, s)
+            taken += int(((cur.seq_lens.astype(np.int64) + B - 1) // B - nb_before).sum())
+            bt2, sl2 = cur.torch_inputs("cuda")[3:]
+            keep.append((bt2, sl2))
+            plan.update(bt2, sl2)
+        o, l = decode_with(plan, cur)
+    assert_all_vs_oracle(cur, o, l, "llama8b after 20 asynchronous updates")
