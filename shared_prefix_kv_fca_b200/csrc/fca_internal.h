@@ -128,6 +128,7 @@ struct fca_plan_s {
     int64_t cap_partials = 0;        // capacity of part_o / part_lse, in rows
     bool async_update = false;       // FCA_PLAN_ASYNC_UPDATE: updates stay on the device; the
                                      // per-request pass reads its item count from sched[2]
+    void* upd_scratch = nullptr;     // temporaries of asynchronous updates
 
     // copies of the inputs
     int32_t* bt = nullptr;           // [R][max_blocks]

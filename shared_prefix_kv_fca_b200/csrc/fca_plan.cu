@@ -969,6 +969,9 @@ struct Arena {
         bytes += align256(std::max<size_t>(count, 1) * sizeof(T));
         return off;
     }
+    void bind(void* base) {
+        for (const Slot& sl : slots) *sl.dst = static_cast<uint8_t*>(base) + sl.off;
+    }
     cudaError_t commit(cudaStream_t stream, void** base) {
         cudaMemPool_t pool = nullptr;
         cudaError_t e = plan_pool(&pool);
@@ -987,6 +990,32 @@ struct TempArena {
     explicit TempArena(cudaStream_t s) : stream(s) {}
     ~TempArena() {
         if (base) cudaFreeAsync(base, stream);
+    }
+};
+
+// Temporaries of one fca_plan_update: from the plan pool for each update, or
+// the plan's own scratch for plans with asynchronous updates.
+struct UpdateTemps {
+    int32_t* valid = nullptr;
+    int32_t* nfull = nullptr;
+    PlanHeader* hdr = nullptr;
+    int32_t* t_nch = nullptr;
+    int32_t* t_chunk = nullptr;
+    int32_t* t_part = nullptr;
+    int32_t* t_item_off = nullptr;
+    int32_t* bin_cursor = nullptr;
+    // lays the arrays out in `ta`; returns the bytes that start at zero
+    size_t layout(Arena& ta, int32_t R, int32_t num_blocks) {
+        ta.add(&valid, num_blocks);
+        ta.add(&hdr, 1);
+        const size_t zero1 = ta.bytes;
+        ta.add(&nfull, R);
+        ta.add(&t_nch, R);
+        ta.add(&t_chunk, R);
+        ta.add(&t_part, R + 1);
+        ta.add(&t_item_off, R + 1);
+        ta.add(&bin_cursor, kBins);
+        return zero1;
     }
 };
 
@@ -1187,6 +1216,12 @@ fca_status plan_build(const int32_t* block_tables, const int32_t* seq_lens, cuda
     wa.add(&P->suffix_items, cap_items);
     wa.add(&P->part_lse, n_part);
     wa.add(&P->part_o, (size_t)n_part * D);
+    if (P->async_update) {
+        UpdateTemps T;
+        Arena probe;
+        T.layout(probe, R, num_blocks);
+        wa.add(reinterpret_cast<uint8_t**>(&P->upd_scratch), probe.bytes);
+    }
     {
         void* base = nullptr;
         if (wa.commit(stream, &base) != cudaSuccess) {
@@ -1277,31 +1312,41 @@ fca_status plan_update(const int32_t* block_tables, const int32_t* seq_lens, cud
     const int32_t R = P->R, max_blocks = P->max_blocks, num_blocks = P->num_blocks;
     const int32_t Hkv = P->Hkv, D = P->D, G = P->G;
 
-    int32_t* valid = nullptr;
-    int32_t* nfull = nullptr;
-    PlanHeader* hdr = nullptr;
-    int32_t* t_nch = nullptr;
-    int32_t* t_chunk = nullptr;
-    int32_t* t_part = nullptr;
-    int32_t* t_item_off = nullptr;
-    int32_t* bin_cursor = nullptr;
+    UpdateTemps T;
     Arena ta;
-    ta.add(&valid, num_blocks);
-    ta.add(&hdr, 1);
-    const size_t zero1 = ta.bytes;
-    ta.add(&nfull, R);
-    ta.add(&t_nch, R);
-    ta.add(&t_chunk, R);
-    ta.add(&t_part, R + 1);
-    ta.add(&t_item_off, R + 1);
-    ta.add(&bin_cursor, kBins);
+    const size_t zero1 = T.layout(ta, R, num_blocks);
+    int32_t* valid = T.valid;
+    int32_t* nfull = T.nfull;
+    PlanHeader* hdr = T.hdr;
+    int32_t* t_nch = T.t_nch;
+    int32_t* t_chunk = T.t_chunk;
+    int32_t* t_part = T.t_part;
+    int32_t* t_item_off = T.t_item_off;
+    int32_t* bin_cursor = T.bin_cursor;
     TempArena tmp(stream);
-    if (ta.commit(stream, &tmp.base) != cudaSuccess) {
-        tmp.base = nullptr;
-        (void)cudaGetLastError();
-        return FCA_ERR_OOM;
+    void* tbase = nullptr;
+    if (P->async_update) {
+        // the plan's own scratch (no allocation, so that the update can be
+        // captured in a CUDA graph along with the decode)
+        ta.bind(P->upd_scratch);
+        tbase = P->upd_scratch;
+    } else {
+        if (ta.commit(stream, &tmp.base) != cudaSuccess) {
+            tmp.base = nullptr;
+            (void)cudaGetLastError();
+            return FCA_ERR_OOM;
+        }
+        tbase = tmp.base;
     }
-    FCA_CK(cudaMemsetAsync(tmp.base, 0, zero1, stream));
+    valid = T.valid;
+    nfull = T.nfull;
+    hdr = T.hdr;
+    t_nch = T.t_nch;
+    t_chunk = T.t_chunk;
+    t_part = T.t_part;
+    t_item_off = T.t_item_off;
+    bin_cursor = T.bin_cursor;
+    FCA_CK(cudaMemsetAsync(tbase, 0, zero1, stream));
     const int64_t cells = (int64_t)R * max_blocks;
     k_validate<<<grid_for(cells, 256), 256, 0, stream>>>(block_tables, max_blocks, seq_lens, R, num_blocks, nfull,
                                                           valid, hdr);
