@@ -13,8 +13,9 @@
 // each behind a lookup of where its rows lie, so it is bound by memory
 // latency and by instructions, not by bandwidth; it is laid out for two
 // rounds of loads per unit of work and few instructions per row:
-//   - a warp takes HB query heads of one (request r, KV head h): grid
-//     (R / 8, Hkv x head blocks), no division but one per warp;
+//   - a warp takes HB query heads of one (request r, KV head h), a unit;
+//     the grid is persistent (3 CTAs of 8 warps per SM), a warp taking
+//     units w, w + all warps, ..., a request's units on neighbouring warps;
 //   - lookup (first round): one lane per entry of the request's chain.  The
 //     planner records where each group partial lies (m_rec, up to kMergeRec),
 //     read together with the request's own-chunk count and first row; deeper
