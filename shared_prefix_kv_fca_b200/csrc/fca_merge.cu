@@ -14,7 +14,7 @@
 // latency and by instructions, not by bandwidth; it is laid out for two
 // rounds of loads per unit of work and few instructions per row:
 //   - a warp takes HB query heads of one (request r, KV head h), a unit;
-//     the grid is persistent (3 CTAs of 8 warps per SM), a warp taking
+//     the grid is persistent (4 CTAs of 8 warps per SM), a warp taking
 //     units w, w + all warps, ..., a request's units on neighbouring warps;
 //   - lookup (first round): one lane per entry of the request's chain.  The
 //     planner records where each group partial lies (m_rec, up to kMergeRec),
@@ -25,8 +25,8 @@
 //     same time, every lane its four columns of the first KK partials'
 //     rows; the maximum and the weight sum of each head take log2(n)
 //     shuffle steps over the n lanes that hold partials; further rows are
-//     read KK at a time.  (HB, KK) = (4, 2) for a few partials a row, (1, 8)
-//     for many.
+//     read KK at a time.  (HB, KK) = (2, 2) for a few partials a row, (1, 8)
+//     for many (64 registers, 4 CTAs of 8 warps per SM).
 // Requests with more than 32 partials, or chains longer than 32 groups, take
 // a per-head loop over batches of 32 partials with a running maximum.
 // Partials with lse = -inf (empty chunks) never contribute: their rows may
@@ -61,7 +61,7 @@ struct MergeArgs {
 namespace {
 
 constexpr int kWarps = 8;       // warps per CTA
-constexpr int kCtasPerSM = 3;   // resident CTAs per SM (the persistent grid)
+constexpr int kCtasPerSM = 4;   // resident CTAs per SM (the persistent grid)
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ int32_t warp_incl_scan(int32_t v, int lane) {
@@ -304,7 +304,7 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_
     const int64_t pairs = (int64_t)P->R * P->Hq;
     const int64_t n_part = (int64_t)P->hdr.n_prefix_partials + P->hdr.n_suffix_partials;
     const bool many = pairs > 0 && n_part > 4 * pairs;
-    const int hb = many ? 1 : 4;
+    const int hb = many ? 1 : 2;
     a.n_hb = (P->G + hb - 1) / hb;
     cudaLaunchConfig_t cfg = {};
     int dev = 0, sms = 148;
@@ -320,8 +320,8 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_
     cfg.attrs = attr;
     cfg.numAttrs = after_pass ? 1 : 0;
     if (P->D == 128)
-        return many ? cudaLaunchKernelEx(&cfg, k_merge<128, 1, 8>, a) : cudaLaunchKernelEx(&cfg, k_merge<128, 4, 2>, a);
-    return many ? cudaLaunchKernelEx(&cfg, k_merge<64, 1, 8>, a) : cudaLaunchKernelEx(&cfg, k_merge<64, 4, 2>, a);
+        return many ? cudaLaunchKernelEx(&cfg, k_merge<128, 1, 8>, a) : cudaLaunchKernelEx(&cfg, k_merge<128, 2, 2>, a);
+    return many ? cudaLaunchKernelEx(&cfg, k_merge<64, 1, 8>, a) : cudaLaunchKernelEx(&cfg, k_merge<64, 2, 2>, a);
 }
 
 }  // namespace fca
