@@ -8,8 +8,9 @@ A step is one pass of the whole hot path -- grouped prefix pass, per-request
 pass, log-sum-exp merge -- over the configuration's synthetic batch, with the
 plan built beforehand (plan time is reported separately).  Inputs are
 resident in HBM; L2 is flushed (256 MiB write) before every timed step.
-Every step is one fca_decode call (the two passes run side by side on
-disjoint SMs, then the merge), timed on the device with CUDA events on the
+Every step is one fca_decode call (the two passes share the SMs, the
+per-request pass taking over each SM the grouped pass frees, then the merge),
+timed on the device with CUDA events on the
 launching stream; ms_per_step is the mean over the K timed steps (max over
 ranks).  The roofline times each pass alone on every SM through its own
 entry point, in a second loop after the timed region.
@@ -488,7 +489,7 @@ def fca_arm(args):
                                                        split_tokens=args.split)
 
     def run_steps(p, n, timed, flush_l2=True):
-        """n whole decode steps (fca_decode: both passes side by side, then the
+        """n whole decode steps (fca_decode: both passes at once, then the
         merge), each bracketed by events on the launching stream."""
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         for i in range(n):

@@ -37,7 +37,7 @@ constexpr size_t kStaticScratchBytes = size_t(64) << 20;
 // Per-SM throughput of the two passes when they run side by side, measured on
 // B200 (K/V bytes a second per SM): the grouped pass streams a group's tokens
 // once per 128-row query tile, the per-request pass its own tokens.  Used to
-// split the SMs between the passes and to size the grouped pass's chunks.
+// choose how many SMs the grouped pass starts on and to size its chunks.
 constexpr double kPrefixGBsPerSM = 18.0;
 constexpr double kSuffixGBsPerSM = 49.0;
 
