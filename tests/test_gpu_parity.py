@@ -761,3 +761,44 @@ def test_plan_update_async_full_size_one_token_steps():
             plan.update(bt2, sl2)
         o, l = decode_with(plan, cur)
     assert_all_vs_oracle(cur, o, l, "llama8b after 20 asynchronous updates")
+
+
+def test_update_and_decode_replayed_as_a_cuda_graph():
+    # one decode step of a kept plan (asynchronous update + decode, the
+    # launch dependencies between the three decode kernels included) captured
+    # once as a CUDA graph; each replay, after the next step's queries and
+    # tables are copied into the captured buffers, decodes that step like
+    # attention over them
+    torch = _torch()
+    import shared_prefix_kv_fca_b200 as fca
+    w0 = fca_workloads.random_small(5, max_requests=24)
+    base, steps = growth_steps(w0, 5, n_steps=3)
+    q, k, v, bt, sl = base.torch_inputs("cuda")
+    bt_d, sl_d = bt.clone(), sl.clone()
+    out = torch.empty_like(q)
+    lse = torch.empty(base.R, base.Hq, dtype=torch.float32, device="cuda")
+    with fca.fca_plan(bt, sl, base.num_blocks, w0.Hq, w0.Hkv, w0.D, min_saved_blocks=0,
+                      async_update=True) as plan:
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):   # one eager step first (the kernels' attributes)
+            plan.update(bt_d, sl_d, cap)
+            fca.fca_decode(q, k, v, plan, out, lse, base.scale, cap)
+        cap.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            plan.update(bt_d, sl_d, cap)
+            fca.fca_decode(q, k, v, plan, out, lse, base.scale, cap)
+        for s, cur in enumerate(steps):
+            q2, _, _, bt2, sl2 = cur.torch_inputs("cuda")   # (same caches, new queries)
+            q.copy_(q2)
+            bt_d.copy_(bt2)
+            sl_d.copy_(sl2)
+            g.replay()
+            torch.cuda.synchronize()
+            assert fca.fca_check_device_status(plan) == 0
+            o_ref, l_ref = oracle.paged_attention(cur.q, cur.k_cache, cur.v_cache, cur.block_tables,
+                                                  cur.seq_lens, cur.scale)
+            assert_close(out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
+                         o_ref, l_ref, f"graph replay step {s + 1}")
+        del g
