@@ -26,7 +26,9 @@
 //     rows; the maximum and the weight sum of each head take log2(n)
 //     shuffle steps over the n lanes that hold partials; further rows are
 //     read KK at a time.  (HB, KK) = (2, 2) for a few partials a row, (1, 8)
-//     for many (64 registers, 4 CTAs of 8 warps per SM).
+//     for many (64 registers, 4 CTAs of 8 warps per SM).  Where G is a power
+//     of two and rows have few partials, a warp takes a whole KV head
+//     instead (merge_kv_unit: one load for every lse of the request).
 // Requests with more than 32 partials, or chains longer than 32 groups, take
 // a per-head loop over batches of 32 partials with a running maximum.
 // Partials with lse = -inf (empty chunks) never contribute: their rows may
@@ -61,7 +63,8 @@ struct MergeArgs {
 namespace {
 
 constexpr int kWarps = 8;       // warps per CTA
-constexpr int kCtasPerSM = 4;   // resident CTAs per SM (the persistent grid)
+constexpr int kCtasPerSM = 4;     // resident CTAs per SM (the persistent grid)
+constexpr int kCtasPerSMKv = 4;   // the same for whole KV heads a warp
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ int32_t warp_incl_scan(int32_t v, int lane) {
@@ -259,6 +262,80 @@ __device__ __forceinline__ void merge_unit(const MergeArgs& a, int32_t r, int32_
     }
 }
 
+// All G query heads of (request r, KV head h), G a power of two, when the
+// request has at most 32 / G partials: lane k G + i holds head i of partial
+// k, so one load gives every lse, and each head's maximum and weight sum take
+// log2(n) shuffle steps over lanes G apart; the rows are then read four heads
+// of one partial at a time (64 registers: 4 CTAs per SM).  Otherwise the unit
+// goes to merge_unit, two heads at a time.
+template <int D>
+__device__ __forceinline__ void merge_kv_unit(const MergeArgs& a, int32_t r, int32_t h, int lane) {
+    constexpr int KK = 1;
+    const int32_t G = a.G;
+    const Entries E = lookup(a, r, h, lane);
+    const int32_t n = E.n;
+    if (!E.wide || n * G > 32) {
+        for (int32_t gq0 = 0; gq0 < G; gq0 += 2) merge_unit<D, 2, 2>(a, r, h, gq0, lane);
+        return;
+    }
+    const int32_t lg = __ffs(G) - 1;   // log2 G
+    const int32_t kl = lane >> lg, il = lane & (G - 1);
+    const int32_t row = partial_row(a, E, h, kl);   // head 0's row of partial kl (lanes kl < n)
+    const float lk = lane < n * G ? __ldg(a.part_lse + row + il) : -INFINITY;
+    const bool cols = lane < D / 4;
+    float4 o[KK][4];
+    auto load_rows = [&](int32_t b0, int32_t k0) {
+#pragma unroll
+        for (int u = 0; u < KK; ++u) {
+            const int32_t ru = __shfl_sync(kFull, row, ((k0 + u) << lg) & 31);
+            const float* src = a.part_o + ((int64_t)ru + b0) * D + lane * 4;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                o[u][j] = (k0 + u < n && b0 + j < G && cols) ? __ldg(reinterpret_cast<const float4*>(src + j * D))
+                                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    load_rows(0, 0);
+    float mx = lk;
+    for (int s = G; s < G * n; s <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, s));
+    const float w = lk == -INFINITY ? 0.f : __expf(lk - mx);
+    float sm = w;
+    for (int s = G; s < G * n; s <<= 1) sm += __shfl_xor_sync(kFull, sm, s);
+    // lanes i < G (partial 0) hold head i's maximum and sum
+    const int32_t q0 = r * a.Hq + h * G;
+    for (int32_t b0 = 0; b0 < G; b0 += 4) {
+        float4 acc[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int32_t k0 = 0; k0 < n; k0 += KK) {
+            if (b0 > 0 || k0 > 0) load_rows(b0, k0);
+#pragma unroll
+            for (int u = 0; u < KK; ++u)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float wu = __shfl_sync(kFull, w, (((k0 + u) << lg) + b0 + j) & 31);
+                    if (k0 + u < n && b0 + j < G && wu > 0.f) fma4(acc[j], wu, o[u][j]);
+                }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float mj = __shfl_sync(kFull, mx, (b0 + j) & 31), lj = __shfl_sync(kFull, sm, (b0 + j) & 31);
+            if (b0 + j < G) store_row<D>(a, q0 + b0 + j, acc[j], mj, lj, lane);
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(32 * kWarps, kCtasPerSMKv) k_merge_kv(MergeArgs a) {
+    dev::pdl_wait();   // (as k_merge)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int32_t n_units = a.R * a.Hkv;
+    for (int32_t u = blockIdx.x * kWarps + warp; u < n_units; u += gridDim.x * kWarps) {
+        const int32_t r = u / a.Hkv;
+        merge_kv_unit<D>(a, r, u - r * a.Hkv, lane);
+    }
+}
+
 template <int D, int HB, int KK>
 __global__ void __launch_bounds__(32 * kWarps, kCtasPerSM) k_merge(MergeArgs a) {
     // launched after a pass with programmatic serialization: its rows are
@@ -304,13 +381,16 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_
     const int64_t pairs = (int64_t)P->R * P->Hq;
     const int64_t n_part = (int64_t)P->hdr.n_prefix_partials + P->hdr.n_suffix_partials;
     const bool many = pairs > 0 && n_part > 4 * pairs;
-    const int hb = many ? 1 : 2;
+    // whole KV heads a warp where G is a power of two (few partials a row)
+    const bool kv = !many && P->G <= 16 && (P->G & (P->G - 1)) == 0;
+    const int hb = many ? 1 : kv ? P->G : 2;
     a.n_hb = (P->G + hb - 1) / hb;
     cudaLaunchConfig_t cfg = {};
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t units = (int64_t)P->R * P->Hkv * a.n_hb;
-    cfg.gridDim = dim3((unsigned)std::min<int64_t>((units + kWarps - 1) / kWarps, (int64_t)sms * kCtasPerSM));
+    cfg.gridDim = dim3((unsigned)std::min<int64_t>((units + kWarps - 1) / kWarps,
+                                                   (int64_t)sms * (kv ? kCtasPerSMKv : kCtasPerSM)));
     cfg.blockDim = dim3(32 * kWarps);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
@@ -320,8 +400,12 @@ cudaError_t launch_merge(const fca_plan_s* P, void* out, float* lse, bool after_
     cfg.attrs = attr;
     cfg.numAttrs = after_pass ? 1 : 0;
     if (P->D == 128)
-        return many ? cudaLaunchKernelEx(&cfg, k_merge<128, 1, 8>, a) : cudaLaunchKernelEx(&cfg, k_merge<128, 2, 2>, a);
-    return many ? cudaLaunchKernelEx(&cfg, k_merge<64, 1, 8>, a) : cudaLaunchKernelEx(&cfg, k_merge<64, 2, 2>, a);
+        return many ? cudaLaunchKernelEx(&cfg, k_merge<128, 1, 8>, a)
+               : kv ? cudaLaunchKernelEx(&cfg, k_merge_kv<128>, a)
+                    : cudaLaunchKernelEx(&cfg, k_merge<128, 2, 2>, a);
+    return many ? cudaLaunchKernelEx(&cfg, k_merge<64, 1, 8>, a)
+           : kv ? cudaLaunchKernelEx(&cfg, k_merge_kv<64>, a)
+                : cudaLaunchKernelEx(&cfg, k_merge<64, 2, 2>, a);
 }
 
 }  // namespace fca
