@@ -220,7 +220,9 @@ fca_status fca_suffix_pass(const void *q, const void *k_cache, const void *v_cac
                            float scale, void *stream);
 fca_status fca_merge_pass(fca_plan_t plan, void *out, float *lse, void *stream);
 
-/* Sizes and byte counts of a plan (HOST struct, filled synchronously). */
+/* Sizes and byte counts of a plan (HOST struct, filled synchronously): of the
+ * plan as built or last updated synchronously (a plan built with
+ * FCA_PLAN_ASYNC_UPDATE keeps the figures of the plan as built). */
 typedef struct fca_plan_stats {
     int32_t num_requests, num_groups, max_depth, num_q_heads, num_kv_heads, head_dim;
     int32_t split_tokens;           /* chunk target of the per-request pass */

@@ -437,6 +437,9 @@ class Plan:
         self.device = device        # CUDA device index the plan belongs to
 
     def stats(self) -> dict:
+        """Sizes and byte counts (fca_plan_get_stats): of the plan as built or
+        last updated synchronously; an asynchronously updated plan keeps the
+        figures of the plan as built."""
         return fca_plan_get_stats(self)
 
     def update(self, block_tables, seq_lens, stream=None) -> None:
