@@ -688,7 +688,9 @@ def fca_arm(args):
             cap = torch.cuda.Stream(dev)
             cap.wait_stream(stream)
             g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=cap):
+            # (thread-local capture: another thread's CUDA calls, a process
+            # group's watchdog for one, do not invalidate it)
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
                 side.wait_stream(cap)
                 with torch.cuda.stream(side):
                     q_d.copy_(q_h, non_blocking=True)
