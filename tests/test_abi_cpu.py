@@ -137,3 +137,12 @@ def test_c_client_links_and_runs(tmp_path, lib):
     assert msg == "block id out of range"
     assert (s_plan, s_dim, no_plan, s_upd, s_self, s_destroy) == ("1", "3", "1", "1", "1", "0")
     assert (mgs, msv, word) == ("2", "32", "-1")
+
+
+def test_binding_constants_match_the_header():
+    # the plan flags the binding passes on are the header's values
+    src = open(os.path.join(ROOT, "include", "fca.h")).read()
+    defines = dict(re.findall(r"^#define\s+(FCA_\w+)\s+\(?([0-9xa-fA-F]+)[uUlL]*", src, flags=re.M))
+    assert int(defines["FCA_PLAN_FLAT"], 0) == fca.FCA_PLAN_FLAT
+    assert int(defines["FCA_PLAN_ASYNC_UPDATE"], 0) == fca.FCA_PLAN_ASYNC_UPDATE
+    assert fca.FCA_PLAN_FLAT & fca.FCA_PLAN_ASYNC_UPDATE == 0
